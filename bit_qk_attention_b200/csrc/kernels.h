@@ -1,0 +1,60 @@
+// Internal launch interface between the C-ABI layer (api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace binattn {
+
+constexpr int kJobPack = 0;  // sign bits + sum |x| per chunk
+constexpr int kJobAmax = 1;  // per-channel max |v| per chunk
+
+struct PrepDims {
+  int64_t BH;
+  int N, d, dp, nchunk;
+};
+
+struct PrepJob {
+  const void* src;  // [BH][N][d] fp16/bf16
+  int kind;
+  uint32_t* bits;   // pack: [BH][N][4]
+  float* part;      // pack: [BH][nchunk]; amax: [BH][nchunk][dp]
+};
+
+struct PrepParams {
+  PrepJob job[3];
+  PrepDims g;
+};
+
+struct FinalizeParams {
+  PrepDims g;
+  int npack;
+  const float* part_mu[2];
+  float* mu[2];
+  const float* part_amax;  // null: no V job
+  float* inv;              // [BH][dp]
+  float* v_scale;          // [BH][d]
+};
+
+struct QuantParams {
+  PrepDims g;
+  const void* v;
+  const float* inv;
+  int8_t* vq;
+};
+
+cudaError_t launch_prep(const PrepParams& p, int dt, int njobs, cudaStream_t s);
+cudaError_t launch_finalize(const FinalizeParams& p, cudaStream_t s);
+cudaError_t launch_quant(const QuantParams& p, int dt, cudaStream_t s);
+
+// Fused attention on packed operands.
+cudaError_t launch_attn_simt(const AttnParams& p, cudaStream_t s);
+bool attn_tc_supported(const AttnParams& p);
+cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t s);
+
+// Device status word of the kernels with bounded waits.
+cudaError_t read_and_clear_device_status(int* value, cudaStream_t s);
+
+}  // namespace binattn

@@ -1,0 +1,184 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on the same seeded
+inputs. Integer work (sign words, V codes, logits) must be bit-exact; the output O must be
+within max-abs 2e-3 and mean-abs 2e-4 of the oracle's fp32 result (fp32 output)."""
+import numpy as np
+import pytest
+
+import oracle
+from util import O_MAX_ABS, assert_o_close, oracle_bias, oracle_forward, oracle_qkv, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+IMPLS = {"simt": 1, "tcgen05": 2}
+
+
+@pytest.fixture(scope="module")
+def ba():
+    import torch
+    assert torch.cuda.is_available(), "needs a CUDA device"
+    from bit_qk_attention_b200 import build
+    build.build()
+    import bit_qk_attention_b200 as mod
+    mod.lib()
+    yield mod
+    mod.set_attention_impl(0)
+
+
+def _dev(w):
+    import torch
+    return w.q.cuda(), w.k.cuda(), w.v.cuda()
+
+
+def _forward(ba, w, impl, out_dtype=None, softmax_scale=0.0, debug_logits=False):
+    import torch
+    ba.set_attention_impl(impl)
+    q, k, v = _dev(w)
+    bias = ba.bias_from_workload(w, q.device)
+    try:
+        res = ba.attention_fwd(q, k, v, bias, softmax_scale=softmax_scale, out_dtype=out_dtype or torch.float32,
+                               debug_logits=debug_logits)
+    except ba.BinAttnError as e:
+        if impl == 2 and e.status == 2:
+            pytest.skip("shape not taken by the tcgen05 kernel")
+        raise
+    torch.cuda.synchronize()
+    assert ba.last_attention_impl() == impl
+    ba.check_device_status()
+    return res
+
+
+# ----------------------------------------------------------------------------- step kernels
+STEP_CONFIGS = ["tiny", "deit_b", "dit256", "dit512", "dit1024", "sweep4096_d128"]
+
+
+@pytest.mark.parametrize("name", STEP_CONFIGS)
+def test_pack_signs_and_mu(ba, name):
+    from bit_qk_attention_b200 import inputs
+    w = inputs.by_name(name)
+    o = oracle.get()
+    for t in (w.q, w.k):
+        bits, mu = ba.pack_signs(t.cuda())
+        x = t.float().numpy()
+        want_bits = o.pack_signs(x)
+        got = bits.cpu().numpy().view(np.uint32)
+        assert np.array_equal(got, want_bits), "sign words differ"
+        want_mu = o.mu(x)
+        np.testing.assert_allclose(mu.cpu().numpy(), want_mu, rtol=3e-6, atol=0)
+
+
+@pytest.mark.parametrize("name", STEP_CONFIGS)
+def test_quant_v(ba, name):
+    from bit_qk_attention_b200 import inputs
+    w = inputs.by_name(name)
+    vq, vs = ba.quant_v(w.v.cuda())
+    want_q, want_s = oracle.get().quant_v(w.v.float().numpy())
+    got_q = vq.cpu().numpy()
+    assert np.array_equal(got_q[..., :w.d], want_q), "V codes differ"
+    assert np.all(got_q[..., w.d:] == 0), "pad columns must be 0"
+    assert np.array_equal(vs.cpu().numpy(), want_s), "V scales differ"
+
+
+# ----------------------------------------------------------------------------- logits
+@pytest.mark.parametrize("impl", list(IMPLS.values()), ids=list(IMPLS))
+@pytest.mark.parametrize("name", ["tiny", "deit_b", "dit256"])
+def test_debug_logits_bit_exact(ba, name, impl):
+    from bit_qk_attention_b200 import inputs
+    w = inputs.by_name(name)
+    _, lg = _forward(ba, w, impl, debug_logits=True)
+    o = oracle.get()
+    q, k, _ = oracle_qkv(w)
+    want = o.logits(o.pack_signs(q), o.pack_signs(k), w.d)
+    assert np.array_equal(lg.cpu().numpy(), want)
+
+
+# ----------------------------------------------------------------------------- forward
+FWD_CONFIGS = [("tiny", None), ("deit_b", None), ("dit256", None), ("dit512", 64), ("dit1024", 48),
+               ("sweep1024_d64", None), ("sweep4096_d64", 48), ("sweep4096_d128", 48),
+               ("sweep16384_d64", 24), ("sweep32768_d64", 16), ("sweep32768_d128", 16)]
+
+
+@pytest.mark.parametrize("impl", list(IMPLS.values()), ids=list(IMPLS))
+@pytest.mark.parametrize("name,nrows", FWD_CONFIGS, ids=[c[0] for c in FWD_CONFIGS])
+def test_forward_parity(ba, name, nrows, impl):
+    from bit_qk_attention_b200 import inputs
+    w = inputs.by_name(name)
+    out = _forward(ba, w, impl).cpu().numpy()
+    rows = None if nrows is None else sample_rows(w.N, nrows, seed=w.N)
+    want = oracle_forward(w, rows=rows)
+    got = out if rows is None else out[:, :, rows]
+    assert_o_close(got, want, f"{name} impl={impl}")
+
+
+EDGE = [  # B, H, N, d, dtype, bias kind, extra
+    (1, 1, 1, 64, "f16", 0, {}), (1, 2, 2, 1, "bf16", 1, {}), (2, 1, 127, 31, "f16", 1, {}),
+    (1, 2, 129, 33, "bf16", 2, {"grid": (3, 43)}), (1, 1, 197, 72, "f16", 2, {"grid": (14, 14), "n_prefix": 1}),
+    (1, 1, 300, 128, "bf16", 0, {}), (2, 3, 255, 64, "f16", 2, {"grid": (2, 127), "n_prefix": 1}),
+    (1, 2, 256, 96, "bf16", 1, {"batch_bias": True}), (2, 2, 128, 16, "f16", 1, {}),
+    (1, 1, 384, 8, "bf16", 0, {}), (1, 2, 200, 100, "f16", 1, {}), (3, 1, 513, 64, "bf16", 1, {"batch_bias": True}),
+]
+
+
+@pytest.mark.parametrize("impl", list(IMPLS.values()), ids=list(IMPLS))
+@pytest.mark.parametrize("case", EDGE, ids=[f"b{c[0]}h{c[1]}n{c[2]}d{c[3]}{c[4]}k{c[5]}" for c in EDGE])
+def test_edge_shapes(ba, case, impl):
+    import torch
+    from bit_qk_attention_b200 import inputs
+    B, H, N, d, dt, kind, extra = case
+    dtype = torch.float16 if dt == "f16" else torch.bfloat16
+    w = inputs.random_case(B, H, N, d, dtype, kind, seed=N * 7 + d, **extra)
+    out, lg = _forward(ba, w, impl, debug_logits=True)
+    assert_o_close(out.cpu().numpy(), oracle_forward(w), f"edge {case}")
+    o = oracle.get()
+    q, k, _ = oracle_qkv(w)
+    assert np.array_equal(lg.cpu().numpy(), o.logits(o.pack_signs(q), o.pack_signs(k), d))
+
+
+@pytest.mark.parametrize("impl", list(IMPLS.values()), ids=list(IMPLS))
+def test_degenerate_inputs(ba, impl):
+    """All-zero q (mu_q = 0: logits reduce to the bias), negative zeros (sign +1), huge
+    magnitudes (alpha ~ 1e3: a near one-hot softmax), and an explicit softmax scale."""
+    import torch
+    from bit_qk_attention_b200 import inputs
+    w = inputs.random_case(2, 2, 150, 64, torch.float16, 1, seed=5)
+    w.q = torch.zeros_like(w.q)
+    assert_o_close(_forward(ba, w, impl).cpu().numpy(), oracle_forward(w), "zero q")
+    w.q = -torch.zeros_like(w.k)
+    assert_o_close(_forward(ba, w, impl).cpu().numpy(), oracle_forward(w), "negative zero q")
+    w2 = inputs.random_case(1, 2, 200, 64, torch.bfloat16, 2, seed=6, grid=(10, 20))
+    w2.q = (w2.q.float() * 90).bfloat16()
+    w2.k = (w2.k.float() * 90).bfloat16()
+    assert_o_close(_forward(ba, w2, impl).cpu().numpy(), oracle_forward(w2), "huge alpha")
+    w3 = inputs.random_case(1, 3, 170, 48, torch.float16, 1, seed=7)
+    assert_o_close(_forward(ba, w3, impl, softmax_scale=0.37).cpu().numpy(),
+                   oracle_forward(w3, softmax_scale=0.37), "explicit scale")
+
+
+@pytest.mark.parametrize("impl", list(IMPLS.values()), ids=list(IMPLS))
+@pytest.mark.parametrize("odt", ["f16", "bf16"])
+def test_output_dtypes(ba, impl, odt):
+    """O stored in fp16/bf16: within the bar plus half an ulp of the stored value."""
+    import torch
+    from bit_qk_attention_b200 import inputs
+    dtype = torch.float16 if odt == "f16" else torch.bfloat16
+    w = inputs.random_case(2, 2, 333, 64, torch.bfloat16, 1, seed=11)
+    out = _forward(ba, w, impl, out_dtype=dtype).float().cpu().numpy()
+    want = oracle_forward(w)
+    ulp = np.float64(2.0 ** -10 if odt == "f16" else 2.0 ** -7)
+    half_ulp = 0.5 * ulp * np.maximum(np.abs(want), 2.0 ** -14) * 2
+    assert np.all(np.abs(out - want) <= O_MAX_ABS + half_ulp)
+
+
+def test_empty_and_errors_on_device(ba):
+    import torch
+    q = torch.zeros((0, 2, 16, 64), dtype=torch.float16, device="cuda")
+    out = ba.attention_fwd(q, q, q)
+    assert out.shape == (0, 2, 16, 64)
+    w = torch.randn((1, 1, 64, 64), device="cuda").half()
+    small = torch.empty(16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(ba.BinAttnError) as ei:
+        ba.attention_fwd(w, w, w, workspace=small)
+    assert ei.value.status == 4
+    wide = torch.zeros((1, 1, 64, 129), dtype=torch.float16, device="cuda")
+    with pytest.raises(ba.BinAttnError) as ei:
+        ba.attention_fwd(wide, wide, wide)
+    assert ei.value.status == 2
