@@ -204,6 +204,7 @@ def pack_signs(x, stream=None) -> Tuple[object, object]:
     bits = torch.empty((B, H, N, 4), dtype=torch.int32, device=x.device)
     mu = torch.empty((B, H), dtype=torch.float32, device=x.device)
     nws = lib().ba_pack_workspace_bytes(B, H, N, d)
+    nws = 0 if nws == ctypes.c_size_t(-1).value else nws
     ws = torch.empty(max(nws, 1), dtype=torch.uint8, device=x.device)
     _check(lib().ba_pack_signs(_ptr(x), _dt(x), B, H, N, d, _ptr(bits), _ptr(mu), _ptr(ws), nws,
                                _stream(stream)), "ba_pack_signs")
@@ -218,6 +219,7 @@ def quant_v(v, stream=None) -> Tuple[object, object]:
     vq = torch.empty((B, H, N, max(v_row_bytes(d), 1)), dtype=torch.int8, device=v.device)
     vs = torch.empty((B, H, d), dtype=torch.float32, device=v.device)
     nws = lib().ba_quant_workspace_bytes(B, H, N, d)
+    nws = 0 if nws == ctypes.c_size_t(-1).value else nws
     ws = torch.empty(max(nws, 1), dtype=torch.uint8, device=v.device)
     _check(lib().ba_quant_v(_ptr(v), _dt(v), B, H, N, d, _ptr(vq), _ptr(vs), _ptr(ws), nws, _stream(stream)),
            "ba_quant_v")
@@ -252,6 +254,8 @@ def attention_fwd(q, k, v, bias: Optional[Bias] = None, softmax_scale: float = 0
     if out is None:
         out = torch.empty((B, H, N, d), dtype=out_dtype or q.dtype, device=q.device)
     nws = lib().ba_workspace_bytes(B, H, N, d)
+    if nws == ctypes.c_size_t(-1).value:  # unsupported size: the call below reports it
+        nws = 0
     if workspace is None:
         workspace = torch.empty(max(nws, 1), dtype=torch.uint8, device=q.device)
     dbg = torch.empty((B, H, N, N), dtype=torch.int32, device=q.device) if debug_logits else None

@@ -119,8 +119,8 @@ WsLayout layout(int B, int H, int N, int d, int what) {
     L.v_scale = take(static_cast<size_t>(g.BH) * d * 4);
   }
   if (what & kWsPack) {
-    L.part_mu_q = take(static_cast<size_t>(g.BH) * g.nchunk * 4);
-    if (what == kWsAll) L.part_mu_k = take(static_cast<size_t>(g.BH) * g.nchunk * 4);
+    L.part_mu_q = take(static_cast<size_t>(g.BH) * g.nchunk * 8);
+    if (what == kWsAll) L.part_mu_k = take(static_cast<size_t>(g.BH) * g.nchunk * 8);
   }
   if (what & kWsQuant) {
     L.part_amax = take(static_cast<size_t>(g.BH) * g.nchunk * g.dp * 4);
@@ -178,11 +178,11 @@ ba_status check_bias(const ba_bias* bz, int N, BiasParams* out) {
   return BA_OK;
 }
 
-ba_status run_pack(const void* x, int dt, const PrepDims& g, uint32_t* bits, float* mu, float* part,
+ba_status run_pack(const void* x, int dt, const PrepDims& g, uint32_t* bits, float* mu, double* part,
                    cudaStream_t s) {
   PrepParams pp{};
   pp.g = g;
-  pp.job[0] = PrepJob{x, kJobPack, bits, part};
+  pp.job[0] = PrepJob{x, kJobPack, bits, part, nullptr};
   pp.job[1] = pp.job[2] = pp.job[0];
   ba_status st = cuda_status(launch_prep(pp, dt, 1, s));
   if (st != BA_OK) return st;
@@ -252,7 +252,7 @@ ba_status ba_pack_signs(const void* x, ba_dtype dt, int B, int H, int N, int d, 
   if (!aligned16(x) || !aligned16(bits) || !aligned16(mu)) return BA_ERR_ALIGNMENT;
   const WsLayout L = layout(B, H, N, d, kWsPack);
   if ((st = check_ws(ws, ws_bytes, L.total)) != BA_OK) return st;
-  return run_pack(x, dt, dims(B, H, N, d), bits, mu, at<float>(ws, L.part_mu_q),
+  return run_pack(x, dt, dims(B, H, N, d), bits, mu, at<double>(ws, L.part_mu_q),
                   static_cast<cudaStream_t>(stream));
 }
 
@@ -270,7 +270,7 @@ ba_status ba_quant_v(const void* v, ba_dtype dt, int B, int H, int N, int d, int
   const PrepDims g = dims(B, H, N, d);
   PrepParams pp{};
   pp.g = g;
-  pp.job[0] = PrepJob{v, kJobAmax, nullptr, at<float>(ws, L.part_amax)};
+  pp.job[0] = PrepJob{v, kJobAmax, nullptr, nullptr, at<float>(ws, L.part_amax)};
   pp.job[1] = pp.job[2] = pp.job[0];
   if ((st = cuda_status(launch_prep(pp, dt, 1, s))) != BA_OK) return st;
   FinalizeParams fp{};
@@ -344,16 +344,16 @@ ba_status ba_attention_fwd(const void* q, const void* k, const void* v, ba_dtype
   // maxima for v.
   PrepParams pp{};
   pp.g = g;
-  pp.job[0] = PrepJob{q, kJobPack, at<uint32_t>(ws, L.bits_q), at<float>(ws, L.part_mu_q)};
-  pp.job[1] = PrepJob{k, kJobPack, at<uint32_t>(ws, L.bits_k), at<float>(ws, L.part_mu_k)};
-  pp.job[2] = PrepJob{v, kJobAmax, nullptr, at<float>(ws, L.part_amax)};
+  pp.job[0] = PrepJob{q, kJobPack, at<uint32_t>(ws, L.bits_q), at<double>(ws, L.part_mu_q), nullptr};
+  pp.job[1] = PrepJob{k, kJobPack, at<uint32_t>(ws, L.bits_k), at<double>(ws, L.part_mu_k), nullptr};
+  pp.job[2] = PrepJob{v, kJobAmax, nullptr, nullptr, at<float>(ws, L.part_amax)};
   if ((st = cuda_status(launch_prep(pp, dt, 3, s))) != BA_OK) return keep(ev, false), st;
   record(ev, 1, s);
   FinalizeParams fp{};
   fp.g = g;
   fp.npack = 2;
-  fp.part_mu[0] = at<float>(ws, L.part_mu_q);
-  fp.part_mu[1] = at<float>(ws, L.part_mu_k);
+  fp.part_mu[0] = at<double>(ws, L.part_mu_q);
+  fp.part_mu[1] = at<double>(ws, L.part_mu_k);
   fp.mu[0] = at<float>(ws, L.mu_q);
   fp.mu[1] = at<float>(ws, L.mu_k);
   fp.part_amax = at<float>(ws, L.part_amax);

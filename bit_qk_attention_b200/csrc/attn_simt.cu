@@ -94,14 +94,16 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(AttnParams p) {
     tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 1));
     tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 2));
     const float m_new = fmaxf(m, tmax);
-    const float c = (m == -CUDART_INF_F) ? 0.0f : expf(m - m_new);
+    // exp(m_old - m_new) and exp(s - m) in double, rounded to fp32: the 8-bit code is then
+    // decided on the same correctly rounded fp32 value the CPU reference uses.
+    const float c = (m == -CUDART_INF_F) ? 0.0f : static_cast<float>(exp(static_cast<double>(m) - m_new));
     float lsum = 0.0f;
 #pragma unroll
     for (int u = 0; u < 32; ++u) {
       const int j = quad + 4 * u;
       int code = 0;
       if (s[u] != -CUDART_INF_F) {
-        const float pf = expf(s[u] - m_new);
+        const float pf = static_cast<float>(exp(static_cast<double>(s[u]) - static_cast<double>(m_new)));
         lsum += pf;
         code = min(255, max(0, __float2int_rn(__fmul_rn(255.0f, pf))));
       }

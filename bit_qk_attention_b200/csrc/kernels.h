@@ -17,10 +17,11 @@ struct PrepDims {
 };
 
 struct PrepJob {
-  const void* src;  // [BH][N][d] fp16/bf16
+  const void* src;   // [BH][N][d] fp16/bf16
   int kind;
-  uint32_t* bits;   // pack: [BH][N][4]
-  float* part;      // pack: [BH][nchunk]; amax: [BH][nchunk][dp]
+  uint32_t* bits;    // pack: [BH][N][4]
+  double* part_sum;  // pack: [BH][nchunk] sums of |x|
+  float* part;       // amax: [BH][nchunk][dp] channel maxima
 };
 
 struct PrepParams {
@@ -31,7 +32,7 @@ struct PrepParams {
 struct FinalizeParams {
   PrepDims g;
   int npack;
-  const float* part_mu[2];
+  const double* part_mu[2];
   float* mu[2];
   const float* part_amax;  // null: no V job
   float* inv;              // [BH][dp]

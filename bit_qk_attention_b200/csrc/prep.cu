@@ -20,13 +20,17 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kMaxIter = 8;  // ceil(kPrepTokens / rows_per_pass) for d/8 <= 16
 
-__device__ __forceinline__ float block_sum(float v, float* sred) {
+// Sum over the CTA in double. Every |x| of a 16-bit input is exact in double and the
+// partial sums stay exact while they are below 2^53 units of the smallest input's ulp, so
+// the result does not depend on the summation order in practice (the CPU reference sums
+// sequentially in double and rounds the mean to fp32 the same way).
+__device__ __forceinline__ double block_sum(double v, double* sred) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (lane == 0) sred[warp] = v;
   __syncthreads();
-  float t = 0.0f;
+  double t = 0.0;
   if (threadIdx.x == 0) {
     for (int w = 0; w < kThreads / 32; ++w) t += sred[w];
   }
@@ -37,7 +41,7 @@ __device__ __forceinline__ float block_sum(float v, float* sred) {
 template <typename T>
 __device__ void prep_pack_vec(const PrepJob& job, const PrepDims& g, int64_t bh, int chunk) {
   __shared__ __align__(16) uint8_t sbits[kPrepTokens][16];
-  __shared__ float sred[kThreads / 32];
+  __shared__ double sred[kThreads / 32];
   const int tok0 = chunk * kPrepTokens;
   const int ntok = min(kPrepTokens, g.N - tok0);
   const int tpr = g.d >> 3;
@@ -52,7 +56,7 @@ __device__ void prep_pack_vec(const PrepJob& job, const PrepDims& g, int64_t bh,
     const int r = r0 + it * rpp;
     if (r0 < rpp && r < ntok) u[it] = ldg_stream(base + (static_cast<int64_t>(r) * g.d + sub * 8) * 2);
   }
-  float acc = 0.0f;
+  double acc = 0.0;
 #pragma unroll
   for (int it = 0; it < kMaxIter; ++it) {
     const int r = r0 + it * rpp;
@@ -63,7 +67,7 @@ __device__ void prep_pack_vec(const PrepJob& job, const PrepDims& g, int64_t bh,
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         byte |= (f[e] < 0.0f ? 1u : 0u) << e;
-        acc += fabsf(f[e]);
+        acc += static_cast<double>(fabsf(f[e]));
       }
       sbits[r][sub] = static_cast<uint8_t>(byte);
     }
@@ -72,8 +76,8 @@ __device__ void prep_pack_vec(const PrepJob& job, const PrepDims& g, int64_t bh,
   if (threadIdx.x < ntok)
     reinterpret_cast<uint4*>(job.bits)[bh * g.N + tok0 + threadIdx.x] =
         reinterpret_cast<const uint4*>(&sbits[0][0])[threadIdx.x];
-  const float tot = block_sum(acc, sred);
-  if (threadIdx.x == 0) job.part[bh * g.nchunk + chunk] = tot;
+  const double tot = block_sum(acc, sred);
+  if (threadIdx.x == 0) job.part_sum[bh * g.nchunk + chunk] = tot;
 }
 
 template <typename T>
@@ -123,20 +127,20 @@ template <typename T>
 __device__ void prep_scalar(const PrepJob& job, const PrepDims& g, int64_t bh, int chunk) {
   __shared__ uint32_t swords[kPrepTokens][kSignWords];
   __shared__ int smax[128];
-  __shared__ float sred[kThreads / 32];
+  __shared__ double sred[kThreads / 32];
   const int tok0 = chunk * kPrepTokens;
   const int ntok = min(kPrepTokens, g.N - tok0);
   for (int e = threadIdx.x; e < kPrepTokens * kSignWords; e += kThreads) (&swords[0][0])[e] = 0u;
   if (threadIdx.x < 128) smax[threadIdx.x] = 0;
   __syncthreads();
   const T* base = reinterpret_cast<const T*>(job.src) + (bh * g.N + tok0) * g.d;
-  float acc = 0.0f;
+  double acc = 0.0;
   for (int e = threadIdx.x; e < ntok * g.d; e += kThreads) {
     const int r = e / g.d, c = e - r * g.d;
     const float f = load1<T>(base + e);
     if (job.kind == kJobPack) {
       if (f < 0.0f) atomicOr(&swords[r][c >> 5], 1u << (c & 31));
-      acc += fabsf(f);
+      acc += static_cast<double>(fabsf(f));
     } else {
       atomicMax(&smax[c], __float_as_int(fabsf(f)));  // non-negative floats order like ints
     }
@@ -146,8 +150,8 @@ __device__ void prep_scalar(const PrepJob& job, const PrepDims& g, int64_t bh, i
     if (threadIdx.x < ntok)
       reinterpret_cast<uint4*>(job.bits)[bh * g.N + tok0 + threadIdx.x] =
           reinterpret_cast<const uint4*>(&swords[0][0])[threadIdx.x];
-    const float tot = block_sum(acc, sred);
-    if (threadIdx.x == 0) job.part[bh * g.nchunk + chunk] = tot;
+    const double tot = block_sum(acc, sred);
+    if (threadIdx.x == 0) job.part_sum[bh * g.nchunk + chunk] = tot;
   } else {
     for (int c = threadIdx.x; c < g.dp; c += kThreads)
       job.part[(bh * g.nchunk + chunk) * g.dp + c] = (c < g.d) ? __int_as_float(smax[c]) : 0.0f;
@@ -177,7 +181,7 @@ __global__ void __launch_bounds__(128) finalize_kernel(FinalizeParams p) {
     for (int j = 0; j < p.npack; ++j) {
       // Fixed-order double sum of the chunk partials.
       double s = 0.0;
-      for (int c = threadIdx.x; c < g.nchunk; c += 32) s += static_cast<double>(p.part_mu[j][bh * g.nchunk + c]);
+      for (int c = threadIdx.x; c < g.nchunk; c += 32) s += p.part_mu[j][bh * g.nchunk + c];
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
       if (threadIdx.x == 0) p.mu[j][bh] = static_cast<float>(s / (static_cast<double>(g.N) * g.d));
