@@ -63,6 +63,7 @@ struct Cfg {
   static constexpr int kNumBars = 6 + 3 * NQ;
   static constexpr int offMisc = offBar + kNumBars * 8;
   static constexpr int kBytes = offMisc + 16;
+  static constexpr int kTabOff = (kBytes + 127) / 128 * 128;
   // Tensor-memory columns of query tile q: S (fp32, 128), P (u8 codes, 32), O (s32, DP).
   __host__ __device__ static constexpr uint32_t tS(int q) { return q * 256; }
   __host__ __device__ static constexpr uint32_t tP(int q) { return q * 256 + 128; }
@@ -136,7 +137,8 @@ __device__ __forceinline__ void expand_signs(uint8_t* dst, const uint4* bits_row
 
 template <int DP, int BK>
 __global__ void __launch_bounds__(Cfg<DP>::kThreads, 1)
-    attn_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmap_v) {
+    attn_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmap_v, int tab_mode, int tsize,
+                   int kmax) {
   using C = Cfg<DP>;
   constexpr int NQ = C::NQ, DQ = C::DQ;
   extern __shared__ uint8_t smem_raw[];
@@ -149,6 +151,9 @@ __global__ void __launch_bounds__(Cfg<DP>::kThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::offBar);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::offMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::offMisc + 4);
+  // Rel-pos table of this CTA's head, staged when it fits: tab_mode 1 = table only,
+  // 2 = table followed by 2*tsize zeros (targets of prefix rows and prefix keys).
+  float* stab = reinterpret_cast<float*>(smem + C::kTabOff);
 
   const int N = p.N, d = p.d;
   const int ctas_per_bh = static_cast<int>(ceil_div(N, BM * NQ));
@@ -177,6 +182,11 @@ __global__ void __launch_bounds__(Cfg<DP>::kThreads, 1)
   }
   if (threadIdx.x < 128)
     sscale[threadIdx.x] = (threadIdx.x < d) ? p.v_scale[bh * d + threadIdx.x] * (1.0f / 255.0f) : 0.0f;
+  if (BK == BA_BIAS_RELPOS2D && tab_mode != 0) {
+    const float* src = p.bias.data + h * static_cast<int64_t>(tsize);
+    const int n = (tab_mode == 2) ? 3 * tsize : tsize;
+    for (int e = threadIdx.x; e < n; e += C::kThreads) stab[e] = (e < tsize) ? __ldg(src + e) : 0.0f;
+  }
   if (warp == 1) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
@@ -209,8 +219,12 @@ __global__ void __launch_bounds__(Cfg<DP>::kThreads, 1)
 #pragma unroll
         for (int u = 0; u < BN / 32; ++u) {
           const int j = lane + 32 * u, tok = t * BN + j;
-          int v = -1;
-          if (tok >= p.bias.n_prefix && tok < N) {
+          // Keys past N read a valid entry (their P is masked); prefix keys read the zeros
+          // after the staged table (or are marked -1 for the general path).
+          int v = (tab_mode == 2) ? -tsize : -1;
+          if (tok >= N) {
+            v = 0;
+          } else if (tok >= p.bias.n_prefix) {
             const int tj = tok - p.bias.n_prefix;
             const int yj = tj / p.bias.grid_w;
             v = yj * W2 + (tj - yj * p.bias.grid_w);
@@ -280,25 +294,36 @@ __global__ void __launch_bounds__(Cfg<DP>::kThreads, 1)
     const int r = w4 * 32 + lane;
     const int i = q0 + q * BM + r;
     const bool row_ok = i < N;
+    const int ic = row_ok ? i : N - 1;  // rows past N read the bias of row N-1 (never stored)
     const uint32_t lane_base = static_cast<uint32_t>(w4 * 32) << 16;
     const uint32_t aS = tmem + lane_base + C::tS(q);
     const uint32_t aP = tmem + lane_base + C::tP(q);
     const uint32_t aO = tmem + lane_base + C::tO(q);
     const float alpha = __fmul_rn(__fmul_rn(p.softmax_scale, p.mu_q[bh]), p.mu_k[bh]);
+    const float2 alpha2 = make_float2(alpha, alpha);
 
-    const float* brow = nullptr;  // dense bias row
-    const float* trow = nullptr;  // rel-pos table of head h
-    int a_i = -1;
-    if (BK == BA_BIAS_DENSE && row_ok) brow = p.bias.data + b * p.bias.batch_stride + (h * N + i) * N;
+    // Bias addressing. Dense: this row of [H][N][N]. Rel-pos: b_ij = tab[a_i - koff_j], where
+    // tab is the head's table (in shared memory when staged, followed by zeros that prefix
+    // rows and prefix keys index into).
+    const float* brow = nullptr;
+    const float* tab = nullptr;
+    int a_i = 0;
+    if (BK == BA_BIAS_DENSE) brow = p.bias.data + b * p.bias.batch_stride + (h * N + ic) * N;
     if (BK == BA_BIAS_RELPOS2D) {
       const int W2 = 2 * p.bias.table_w - 1;
-      trow = p.bias.data + h * static_cast<int64_t>(2 * p.bias.table_h - 1) * W2;
-      if (row_ok && i >= p.bias.n_prefix) {
-        const int ti = i - p.bias.n_prefix;
+      tab = (tab_mode != 0) ? stab : p.bias.data + h * static_cast<int64_t>(2 * p.bias.table_h - 1) * W2;
+      if (ic >= p.bias.n_prefix) {
+        const int ti = ic - p.bias.n_prefix;
         const int yi = ti / p.bias.grid_w;
         a_i = (yi + p.bias.table_h - 1) * W2 + (ti - yi * p.bias.grid_w) + p.bias.table_w - 1;
+      } else {
+        a_i = (tab_mode == 2) ? tsize + kmax : -1;  // prefix row: zeros (or the slow path)
       }
     }
+    // Fast path: full key blocks, no debug output, aligned dense rows, prefix handled by zeros.
+    const bool fast_ok = (p.dbg_logits == nullptr) &&
+                         (BK != BA_BIAS_DENSE || ((N & 3) == 0 && (p.bias.batch_stride & 3) == 0)) &&
+                         (BK != BA_BIAS_RELPOS2D || p.bias.n_prefix == 0 || tab_mode == 2);
 
     float m = -CUDART_INF_F, l = 0.0f;
     float of[DP];
@@ -320,38 +345,90 @@ __global__ void __launch_bounds__(Cfg<DP>::kThreads, 1)
       tc_fence_after();
       const int* ko = koff + s * BN;
 
-      auto bias_of = [&](int j) -> float {
-        if (BK == BA_BIAS_DENSE) return row_ok ? __ldg(brow + t * BN + j) : 0.0f;
-        if (BK == BA_BIAS_RELPOS2D) {
-          const int kj = ko[j];
-          return (a_i >= 0 && kj >= 0) ? __ldg(trow + (a_i - kj)) : 0.0f;
-        }
-        return 0.0f;
-      };
-
-      // Pass 1: block max of s = alpha * x + b.
-      float tmax = -CUDART_INF_F;
+      // Pass 1: s = alpha * x + b written back over S in TMEM; block max.
+      float mx0 = -CUDART_INF_F, mx1 = -CUDART_INF_F;
+      if (fast_ok && nk == BN) {
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t x[32];
-        tmem_ld32(aS + 32 * c, x);
-        tmem_ld_wait32(x);
+        for (int c = 0; c < BN / 32; ++c) {
+          float bv[32];
+          if (BK == BA_BIAS_DENSE) {
+            const float4* src = reinterpret_cast<const float4*>(brow + t * BN + 32 * c);
 #pragma unroll
-        for (int u = 0; u < 32; ++u) {
-          const int j = 32 * c + u;
-          if (j < nk) {
-            const float xf = __uint_as_float(x[u]);
-            tmax = fmaxf(tmax, __fmaf_rn(alpha, xf, bias_of(j)));
-            if (p.dbg_logits != nullptr && row_ok)
-              p.dbg_logits[(bh * N + i) * N + t * BN + j] = __float2int_rn(xf);
+            for (int k4 = 0; k4 < 8; ++k4) {
+              const float4 v4 = __ldg(src + k4);
+              bv[4 * k4] = v4.x; bv[4 * k4 + 1] = v4.y; bv[4 * k4 + 2] = v4.z; bv[4 * k4 + 3] = v4.w;
+            }
+          } else if (BK == BA_BIAS_RELPOS2D) {
+            const int4* kv = reinterpret_cast<const int4*>(ko + 32 * c);
+#pragma unroll
+            for (int k4 = 0; k4 < 8; ++k4) {
+              const int4 o4 = kv[k4];
+              bv[4 * k4] = tab[a_i - o4.x];
+              bv[4 * k4 + 1] = tab[a_i - o4.y];
+              bv[4 * k4 + 2] = tab[a_i - o4.z];
+              bv[4 * k4 + 3] = tab[a_i - o4.w];
+            }
+          } else {
+#pragma unroll
+            for (int u = 0; u < 32; ++u) bv[u] = 0.0f;
           }
+          uint32_t x[32];
+          tmem_ld32(aS + 32 * c, x);
+          tmem_ld_wait32(x);
+#pragma unroll
+          for (int k = 0; k < 16; ++k) {
+            const float2 s2 = __ffma2_rn(alpha2, make_float2(__uint_as_float(x[2 * k]), __uint_as_float(x[2 * k + 1])),
+                                         make_float2(bv[2 * k], bv[2 * k + 1]));
+            x[2 * k] = __float_as_uint(s2.x);
+            x[2 * k + 1] = __float_as_uint(s2.y);
+            if (k & 1)
+              mx1 = fmax3(mx1, s2.x, s2.y);
+            else
+              mx0 = fmax3(mx0, s2.x, s2.y);
+          }
+          tmem_st32(aS + 32 * c, x);
+        }
+      } else {
+        // General path: a partial last block, prefix tokens without zero padding, unaligned
+        // dense rows, or the debug logits.
+        auto bias_of = [&](int j) -> float {
+          if (BK == BA_BIAS_DENSE) return __ldg(brow + t * BN + j);
+          if (BK == BA_BIAS_RELPOS2D) {
+            const int kj = ko[j];
+            return (a_i >= 0 && kj >= 0) ? tab[a_i - kj] : 0.0f;
+          }
+          return 0.0f;
+        };
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t x[32];
+          tmem_ld32(aS + 32 * c, x);
+          tmem_ld_wait32(x);
+#pragma unroll
+          for (int u = 0; u < 32; ++u) {
+            const int j = 32 * c + u;
+            float sv = -CUDART_INF_F;
+            if (j < nk) {
+              const float xf = __uint_as_float(x[u]);
+              sv = __fmaf_rn(alpha, xf, bias_of(j));
+              if (p.dbg_logits != nullptr && row_ok)
+                p.dbg_logits[(bh * N + i) * N + t * BN + j] = __float2int_rn(xf);
+            }
+            mx0 = fmaxf(mx0, sv);
+            x[u] = __float_as_uint(sv);
+          }
+          tmem_st32(aS + 32 * c, x);
         }
       }
-      const float m_new = fmaxf(m, tmax);
-      const float mL = m_new * kLog2e;
+      const float m_new = fmaxf(m, fmaxf(mx0, mx1));
+      tmem_st_wait();
 
-      // Pass 2: P~ = 2^((s - m) log2 e), row sum, 8-bit codes -> TMEM.
-      float lt = 0.0f;
+      // Pass 2: P~ = 2^((s - m) log2 e) (masked keys hold s = -inf: P~ = 0), row sum, codes -> TMEM.
+      const float2 negm2 = make_float2(-m_new, -m_new);
+      const float2 log2e2 = make_float2(kLog2e, kLog2e);
+      const float2 c255 = make_float2(255.0f, 255.0f);
+      const float2 magic2 = make_float2(12582912.0f, 12582912.0f);
+      float2 lt2 = make_float2(0.0f, 0.0f);
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         uint32_t x[32];
@@ -362,22 +439,24 @@ __global__ void __launch_bounds__(Cfg<DP>::kThreads, 1)
         for (int w = 0; w < 8; ++w) {
           uint32_t y[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int u = 4 * w + e, j = 32 * c + u;
-            float pf = 0.0f;
-            if (j < nk) {
-              const float sv = __fmaf_rn(alpha, __uint_as_float(x[u]), bias_of(j));
-              pf = ex2_approx(__fmaf_rn(sv, kLog2e, -mL));
-            }
-            lt += pf;
+          for (int e2 = 0; e2 < 2; ++e2) {
+            const int u = 4 * w + 2 * e2;
+            // s - m first (exact near the max), then the scale to base 2.
+            const float2 t2 = __fmul2_rn(
+                __fadd2_rn(make_float2(__uint_as_float(x[u]), __uint_as_float(x[u + 1])), negm2), log2e2);
+            const float2 p2 = make_float2(ex2_approx(t2.x), ex2_approx(t2.y));
+            lt2 = __fadd2_rn(lt2, p2);
             // 255 P~ + 1.5 * 2^23: one rounding to the nearest integer (ties to even); the
             // integer sits in the low byte of the result (P~ <= 1).
-            y[e] = __float_as_uint(__fmaf_rn(pf, 255.0f, 12582912.0f));
+            const float2 y2 = __ffma2_rn(p2, c255, magic2);
+            y[2 * e2] = __float_as_uint(y2.x);
+            y[2 * e2 + 1] = __float_as_uint(y2.y);
           }
           pk[w] = __byte_perm(__byte_perm(y[0], y[1], 0x0040), __byte_perm(y[2], y[3], 0x0040), 0x5410);
         }
         tmem_st8(aP + 8 * c, pk);
       }
+      const float lt = lt2.x + lt2.y;
       const float ct = (m == -CUDART_INF_F) ? 0.0f : ex2_approx((m - m_new) * kLog2e);
       l = l * ct + lt;
       const bool flush = (t > 0) && (m_new > m);
@@ -452,19 +531,33 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+constexpr int kMaxSmem = 227 * 1024;
+
 template <int DP, int BK>
 cudaError_t launch_dp_bk(const AttnParams& p, const CUtensorMap& tm, cudaStream_t s) {
   using C = Cfg<DP>;
+  int tab_mode = 0, tsize = 0, kmax = 0;
+  if (BK == BA_BIAS_RELPOS2D) {
+    tsize = (2 * p.bias.table_h - 1) * (2 * p.bias.table_w - 1);
+    kmax = (p.bias.grid_h - 1) * (2 * p.bias.table_w - 1) + p.bias.grid_w - 1;
+    const int64_t room = kMaxSmem - 1024 - C::kTabOff;
+    if (p.bias.n_prefix > 0 && 3ll * tsize * 4 <= room)
+      tab_mode = 2;
+    else if (static_cast<int64_t>(tsize) * 4 <= room)
+      tab_mode = 1;
+  }
+  const int tab_bytes = tab_mode == 0 ? 0 : (tab_mode == 2 ? 3 : 1) * tsize * 4;
   // At least 116 KB of shared memory per CTA keeps one CTA per SM (it owns all 512 TMEM columns).
-  const int smem = (C::kBytes + 1024 > 116 * 1024) ? C::kBytes + 1024 : 116 * 1024;
-  static bool configured = false;
-  if (!configured) {
+  int smem = C::kTabOff + tab_bytes + 1024;
+  if (smem < 116 * 1024) smem = 116 * 1024;
+  static int configured = 0;
+  if (smem > configured) {
     cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<DP, BK>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    configured = true;
+    configured = smem;
   }
   const int64_t grid = static_cast<int64_t>(p.B) * p.H * ceil_div(p.N, BM * C::NQ);
-  attn_tc_kernel<DP, BK><<<static_cast<unsigned>(grid), C::kThreads, smem, s>>>(p, tm);
+  attn_tc_kernel<DP, BK><<<static_cast<unsigned>(grid), C::kThreads, smem, s>>>(p, tm, tab_mode, tsize, kmax);
   return cudaGetLastError();
 }
 
