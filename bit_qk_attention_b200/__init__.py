@@ -58,6 +58,8 @@ SIGNATURES = {
                                      _I, _P, _P]),
     "ba_attention_fwd": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, ctypes.POINTER(CBias), _F, _P, _I, _P, _SZ,
                               _P, _P]),
+    "ba_attention_fwd_noalloc": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, ctypes.POINTER(CBias), _F, _P, _I, _P,
+                                      _P]),
     "ba_set_attention_impl": (_I, [_I]),
     "ba_get_attention_impl": (_I, []),
     "ba_last_attention_impl": (_I, []),

@@ -137,6 +137,28 @@ ba_status ba_attention_fwd(const void* q, const void* k, const void* v, ba_dtype
                            void* stream);
 
 /*
+ * ba_attention_fwd without a caller-supplied workspace (the paper has no counterpart; this
+ * is a deployment convenience). For callers that cannot allocate device memory: a plugin that
+ * is handed only its input and output buffers, or a runtime that fixes all device memory at
+ * start-up and forbids cudaMalloc afterwards (it can synchronize the device and bypasses the
+ * host's allocator). The workspace comes from a fixed array of BA_NOALLOC_SCRATCH_BYTES in the
+ * library's device memory, held by every GPU that loads the library until the process exits.
+ *   - Arguments as ba_attention_fwd, minus ws / ws_bytes.
+ *   - Problems with ba_workspace_bytes(B,H,N,d) > BA_NOALLOC_SCRATCH_BYTES return
+ *     BA_ERR_WORKSPACE before anything is launched.
+ *   - All calls share the array: calls that can overlap on the GPU (unordered streams) race
+ *     and must be ordered by the caller. Its contents persist between calls; none of it needs
+ *     to start at zero.
+ *   - The first call on each device looks up the array's device address (and caches it);
+ *     make that first call before any stream capture.
+ *   - Allocates nothing: no cudaMalloc, cudaFree or other allocating routine.
+ */
+#define BA_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+ba_status ba_attention_fwd_noalloc(const void* q, const void* k, const void* v, ba_dtype dt, int B, int H,
+                                   int N, int d, const ba_bias* bias, float softmax_scale, void* o,
+                                   ba_dtype o_dt, int32_t* dbg_logits, void* stream);
+
+/*
  * Kernel choice for the fused step, process-wide: 0 = automatic (the tcgen05 tensor-core
  * kernel where it supports the shape, else the CUDA-core kernel), 1 = the CUDA-core kernel,
  * 2 = the tcgen05 kernel (BA_ERR_UNSUPPORTED for shapes it does not take).
