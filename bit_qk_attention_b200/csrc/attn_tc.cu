@@ -54,28 +54,37 @@ struct Cfg {
   static constexpr int kQBytes = BM * DQ;
   static constexpr int kKBytes = BN * DQ;
   static constexpr int kVBytes = BN * DP;
+  static constexpr int kStages = 4;                 // K/V pipeline depth
   static constexpr int offQ = 0;
   static constexpr int offK = offQ + NQ * kQBytes;
-  static constexpr int offV = offK + 2 * kKBytes;
-  static constexpr int offKoff = offV + 2 * kVBytes;
-  static constexpr int offScale = offKoff + 2 * BN * 4;
+  static constexpr int offV = offK + kStages * kKBytes;
+  static constexpr int offKoff = offV + kStages * kVBytes;
+  static constexpr int offScale = offKoff + kStages * BN * 4;
   static constexpr int offBar = offScale + 128 * 4;
-  static constexpr int kNumBars = 6 + 3 * NQ;
+  static constexpr int kNumBars = 2 * kStages + 2 + 3 * NQ;
   static constexpr int offMisc = offBar + kNumBars * 8;
   static constexpr int kBytes = offMisc + 16;
   static constexpr int kTabOff = (kBytes + 127) / 128 * 128;
-  // Tensor-memory columns of query tile q: S (fp32, 128), P (u8 codes, 32), O (s32, DP).
+  // Tensor-memory columns of query tile q: S (fp32, 128 columns; the softmax overwrites it
+  // with s and then its first 32 columns with the u8 codes P — the MMAs of one CTA run in
+  // issue order, so P.V reads P before the next QK rewrites S), O (the s32 P.V accumulator,
+  // DP) and F (the fp32 running output, DP).
   __host__ __device__ static constexpr uint32_t tS(int q) { return q * 256; }
-  __host__ __device__ static constexpr uint32_t tP(int q) { return q * 256 + 128; }
-  __host__ __device__ static constexpr uint32_t tO(int q) { return q * 256 + 160; }
-  static_assert(tO(NQ - 1) + DP <= 512, "tensor memory budget");
+  __host__ __device__ static constexpr uint32_t tP(int q) { return q * 256; }
+  __host__ __device__ static constexpr uint32_t tO(int q) { return q * 256 + 128; }
+  __host__ __device__ static constexpr uint32_t tF(int q) { return q * 256 + 128 + DP; }
+  static_assert(tF(NQ - 1) + DP <= 512, "tensor memory budget");
 };
 
-// Barrier slots.
-enum { kKvFull = 0, kKvEmpty = 2, kQFull = 4, kDrain = 5, kSFull = 6 };
-template <int NQ> struct Bars {
-  __host__ __device__ static constexpr int pfull(int q) { return kSFull + NQ + q; }
-  __host__ __device__ static constexpr int odone(int q) { return kSFull + 2 * NQ + q; }
+// Barrier slots: kv_full[S], kv_empty[S], q_full, drain, s_full[NQ], p_full[NQ], o_done[NQ].
+template <int S, int NQ> struct Bars {
+  __host__ __device__ static constexpr int kvfull(int s) { return s; }
+  __host__ __device__ static constexpr int kvempty(int s) { return S + s; }
+  __host__ __device__ static constexpr int qfull() { return 2 * S; }
+  __host__ __device__ static constexpr int drain() { return 2 * S + 1; }
+  __host__ __device__ static constexpr int sfull(int q) { return 2 * S + 2 + q; }
+  __host__ __device__ static constexpr int pfull(int q) { return 2 * S + 2 + NQ + q; }
+  __host__ __device__ static constexpr int odone(int q) { return 2 * S + 2 + 2 * NQ + q; }
 };
 
 // Waits for the phase of `bar` with the given parity. Gives up after kTimeoutNs (recording the
@@ -107,30 +116,77 @@ __device__ __forceinline__ uint32_t channel_mask(int c0, int d) {
   return n >= 4 ? 0xffffffffu : (n <= 0 ? 0u : ((1u << (8 * n)) - 1u));
 }
 
-// 1-bit sign rows -> fp8 e4m3 +-1 (bit 1 = negative) in the K-major no-swizzle core-matrix
-// layout: byte (row r, channel c) at (c/16)*2048 + r*16 + c%16. Channels >= d and rows >= N
-// are 0 so they add nothing to the dot products.
+// One 1-bit sign row -> fp8 e4m3 +-1 (bit 1 = negative) in the K-major no-swizzle core-matrix
+// layout: byte (row r, channel c) at (c/16)*2048 + r*16 + c%16. Channels >= d, and rows past
+// the end (ok = false), are 0 so they add nothing to the dot products.
 template <int DQ>
-__device__ __forceinline__ void expand_signs(uint8_t* dst, const uint4* bits_rows, int row0, int N, int d,
-                                             int lane) {
+__device__ __forceinline__ void expand_row(uint8_t* dst, const uint4& b, bool ok, int r, int d) {
+  const uint32_t w[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
-  for (int u = 0; u < BM / 32; ++u) {
-    const int r = lane + 32 * u;
-    const int tok = row0 + r;
-    const bool ok = tok < N;
-    const uint4 b = ok ? bits_rows[tok] : make_uint4(0u, 0u, 0u, 0u);
-    const uint32_t w[4] = {b.x, b.y, b.z, b.w};
+  for (int kc = 0; kc < DQ / 16; ++kc) {
+    const uint32_t bits16 = (w[kc >> 1] >> (16 * (kc & 1))) & 0xffffu;
+    uint32_t o[4];
 #pragma unroll
-    for (int kc = 0; kc < DQ / 16; ++kc) {
-      const uint32_t bits16 = (w[kc >> 1] >> (16 * (kc & 1))) & 0xffffu;
-      uint32_t o[4];
+    for (int g = 0; g < 4; ++g) {
+      const uint32_t nib = (bits16 >> (4 * g)) & 0xfu;
+      const uint32_t val = ((nib * 0x10204080u) & 0x80808080u) | 0x38383838u;
+      o[g] = ok ? (val & channel_mask(16 * kc + 4 * g, d)) : 0u;
+    }
+    *reinterpret_cast<uint4*>(dst + kc * 2048 + r * 16) = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+// Bias variants of the kernel: BA_BIAS_NONE, BA_BIAS_DENSE, BA_BIAS_RELPOS2D with the head's
+// table staged in shared memory, and kRelposGlobal with the table read from global memory.
+constexpr int kRelposGlobal = 3;
+__host__ __device__ constexpr bool is_relpos(int bk) { return bk == BA_BIAS_RELPOS2D || bk == kRelposGlobal; }
+
+// Fast path of pass 1 for one 32-key block of one row: bias (dense row, or rel-pos table in
+// shared or global memory), s = alpha * x + b in place, running maxima. PARTIAL masks keys
+// at or past nk to -inf.
+template <int BK, bool PARTIAL>
+__device__ __forceinline__ void fast_block(uint32_t (&x)[32], int c, int nk, float2 alpha2, const float* brow_t,
+                                           uint32_t ko_s, uint32_t tb, const float* grow, int tab_mode,
+                                           float (&mx)[4]) {
 #pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        const uint32_t nib = (bits16 >> (4 * g)) & 0xfu;
-        const uint32_t val = ((nib * 0x10204080u) & 0x80808080u) | 0x38383838u;
-        o[g] = ok ? (val & channel_mask(16 * kc + 4 * g, d)) : 0u;
+  for (int g = 0; g < 4; ++g) {
+    float bv[8];
+    if (BK == BA_BIAS_DENSE) {
+      const float4* src = reinterpret_cast<const float4*>(brow_t + 32 * c + 8 * g);
+      const float4 v0 = __ldg(src), v1 = __ldg(src + 1);
+      bv[0] = v0.x; bv[1] = v0.y; bv[2] = v0.z; bv[3] = v0.w;
+      bv[4] = v1.x; bv[5] = v1.y; bv[6] = v1.z; bv[7] = v1.w;
+    } else if (is_relpos(BK)) {
+      const int4 o0 = lds_s32x4(ko_s + 4u * (32 * c + 8 * g));
+      const int4 o1 = lds_s32x4(ko_s + 4u * (32 * c + 8 * g + 4));
+      if (BK == BA_BIAS_RELPOS2D) {
+        bv[0] = lds_f32(tb - o0.x); bv[1] = lds_f32(tb - o0.y);
+        bv[2] = lds_f32(tb - o0.z); bv[3] = lds_f32(tb - o0.w);
+        bv[4] = lds_f32(tb - o1.x); bv[5] = lds_f32(tb - o1.y);
+        bv[6] = lds_f32(tb - o1.z); bv[7] = lds_f32(tb - o1.w);
+      } else {
+        bv[0] = __ldg(grow - (o0.x >> 2)); bv[1] = __ldg(grow - (o0.y >> 2));
+        bv[2] = __ldg(grow - (o0.z >> 2)); bv[3] = __ldg(grow - (o0.w >> 2));
+        bv[4] = __ldg(grow - (o1.x >> 2)); bv[5] = __ldg(grow - (o1.y >> 2));
+        bv[6] = __ldg(grow - (o1.z >> 2)); bv[7] = __ldg(grow - (o1.w >> 2));
       }
-      *reinterpret_cast<uint4*>(dst + kc * 2048 + r * 16) = make_uint4(o[0], o[1], o[2], o[3]);
+    } else {
+#pragma unroll
+      for (int u = 0; u < 8; ++u) bv[u] = 0.0f;
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int u = 8 * g + 2 * k;
+      const float2 s2 = __ffma2_rn(alpha2, make_float2(__uint_as_float(x[u]), __uint_as_float(x[u + 1])),
+                                   make_float2(bv[2 * k], bv[2 * k + 1]));
+      float sx = s2.x, sy = s2.y;
+      if (PARTIAL) {
+        if (32 * c + u >= nk) sx = -CUDART_INF_F;
+        if (32 * c + u + 1 >= nk) sy = -CUDART_INF_F;
+      }
+      x[u] = __float_as_uint(sx);
+      x[u + 1] = __float_as_uint(sy);
+      mx[k] = fmax3(mx[k], sx, sy);
     }
   }
 }
@@ -140,7 +196,8 @@ __global__ void __launch_bounds__(Cfg<DP>::kThreads, 1)
     attn_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmap_v, int tab_mode, int tsize,
                    int kmax) {
   using C = Cfg<DP>;
-  constexpr int NQ = C::NQ, DQ = C::DQ;
+  constexpr int NQ = C::NQ, DQ = C::DQ, S = C::kStages;
+  using Bar = Bars<S, NQ>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem + C::offQ;
@@ -164,16 +221,17 @@ __global__ void __launch_bounds__(Cfg<DP>::kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    mbar_init(&bars[kKvFull + 0], 2);
-    mbar_init(&bars[kKvFull + 1], 2);
-    mbar_init(&bars[kKvEmpty + 0], 1);
-    mbar_init(&bars[kKvEmpty + 1], 1);
-    mbar_init(&bars[kQFull], 1);
-    mbar_init(&bars[kDrain], 1);
+    for (int st = 0; st < C::kStages; ++st) {
+      // kv_full: the V copy's expect_tx arrival + warp 0 (key offsets) + the two expanding warps.
+      mbar_init(&bars[Bar::kvfull(st)], 4);
+      mbar_init(&bars[Bar::kvempty(st)], 1);
+    }
+    mbar_init(&bars[Bar::qfull()], 2);
+    mbar_init(&bars[Bar::drain()], 1);
     for (int q = 0; q < NQ; ++q) {
-      mbar_init(&bars[kSFull + q], 1);
-      mbar_init(&bars[Bars<NQ>::pfull(q)], 4);
-      mbar_init(&bars[Bars<NQ>::odone(q)], 1);
+      mbar_init(&bars[Bar::sfull(q)], 1);
+      mbar_init(&bars[Bar::pfull(q)], 4);
+      mbar_init(&bars[Bar::odone(q)], 1);
     }
     *abort_flag = 0;
     mbar_fence_init();
@@ -182,7 +240,7 @@ __global__ void __launch_bounds__(Cfg<DP>::kThreads, 1)
   }
   if (threadIdx.x < 128)
     sscale[threadIdx.x] = (threadIdx.x < d) ? p.v_scale[bh * d + threadIdx.x] * (1.0f / 255.0f) : 0.0f;
-  if (BK == BA_BIAS_RELPOS2D && tab_mode != 0) {
+  if (is_relpos(BK) && tab_mode != 0) {
     const float* src = p.bias.data + h * static_cast<int64_t>(tsize);
     const int n = (tab_mode == 2) ? 3 * tsize : tsize;
     for (int e = threadIdx.x; e < n; e += C::kThreads) stab[e] = (e < tsize) ? __ldg(src + e) : 0.0f;
@@ -197,25 +255,18 @@ __global__ void __launch_bounds__(Cfg<DP>::kThreads, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    const uint4* qrows = reinterpret_cast<const uint4*>(p.bits_q) + bh * N;
-    const uint4* krows = reinterpret_cast<const uint4*>(p.bits_k) + bh * N;
-    for (int q = 0; q < NQ; ++q) expand_signs<DQ>(sQ + q * C::kQBytes, qrows, q0 + q * BM, N, d, lane);
-    fence_proxy_async_smem();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&bars[kQFull]);
+    // ------------------------------------------------------------ producer: V blocks, key offsets
     const int W2 = 2 * p.bias.table_w - 1;
     int issued = 0;
     for (int t = 0; t < T; ++t) {
-      const int s = t & 1;
-      if (t >= 2 && !wait_warp(&bars[kKvEmpty + s], ((t >> 1) - 1) & 1, abort_flag)) break;
+      const int st = t % S;
+      if (t >= S && !wait_warp(&bars[Bar::kvempty(st)], ((t / S) - 1) & 1, abort_flag)) break;
       issued = t + 1;
       if (lane == 0) {
-        mbar_arrive_expect_tx(&bars[kKvFull + s], C::kVBytes);
-        tma_load_4d(sV + s * C::kVBytes, &tmap_v, &bars[kKvFull + s], 0, t * BN, 0, static_cast<int>(bh));
+        mbar_arrive_expect_tx(&bars[Bar::kvfull(st)], C::kVBytes);
+        tma_load_4d(sV + st * C::kVBytes, &tmap_v, &bars[Bar::kvfull(st)], 0, t * BN, 0, static_cast<int>(bh));
       }
-      expand_signs<DQ>(sK + s * C::kKBytes, krows, t * BN, N, d, lane);
-      if (BK == BA_BIAS_RELPOS2D) {
+      if (is_relpos(BK)) {
 #pragma unroll
         for (int u = 0; u < BN / 32; ++u) {
           const int j = lane + 32 * u, tok = t * BN + j;
@@ -229,17 +280,65 @@ __global__ void __launch_bounds__(Cfg<DP>::kThreads, 1)
             const int yj = tj / p.bias.grid_w;
             v = yj * W2 + (tj - yj * p.bias.grid_w);
           }
-          koff[s * BN + j] = v;
+          koff[st * BN + j] = 4 * v;  // byte offset into the staged table
         }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[Bar::kvfull(st)]);
+    }
+    // Leave no TMA copy in flight: wait (bounded, even after an abort) for the stages this
+    // warp filled last.
+    for (int t = (issued > S ? issued - S : 0); t < issued; ++t)
+      wait_bounded(&bars[Bar::kvfull(t % S)], (t / S) & 1, abort_flag, false);
+  } else if (warp == 2 || warp == 3) {
+    // ------------------------------------------------------------ producer: sign expansion
+    // Warp 2 expands rows 0..63 and warp 3 rows 64..127 of every Q tile and K block. The
+    // sign rows of the next block are loaded into registers before this block is written.
+    const int half = warp - 2;
+    const uint4* qrows = reinterpret_cast<const uint4*>(p.bits_q) + bh * N;
+    const uint4* krows = reinterpret_cast<const uint4*>(p.bits_k) + bh * N;
+    const uint4 zero4 = make_uint4(0u, 0u, 0u, 0u);
+    for (int q = 0; q < NQ; ++q) {
+      uint4 b[2];
+      bool ok[2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int row = q0 + q * BM + 64 * half + lane + 32 * u;
+        ok[u] = row < N;
+        b[u] = ok[u] ? __ldg(qrows + row) : zero4;
+      }
+#pragma unroll
+      for (int u = 0; u < 2; ++u) expand_row<DQ>(sQ + q * C::kQBytes, b[u], ok[u], 64 * half + lane + 32 * u, d);
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&bars[Bar::qfull()]);
+    uint4 nb[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int row = 64 * half + lane + 32 * u;
+      nb[u] = row < N ? __ldg(krows + row) : zero4;
+    }
+    for (int t = 0; t < T; ++t) {
+      const int st = t % S;
+      const uint4 cb[2] = {nb[0], nb[1]};
+      if (t + 1 < T) {
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int row = (t + 1) * BN + 64 * half + lane + 32 * u;
+          nb[u] = row < N ? __ldg(krows + row) : zero4;
+        }
+      }
+      if (t >= S && !wait_warp(&bars[Bar::kvempty(st)], ((t / S) - 1) & 1, abort_flag)) break;
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int r = 64 * half + lane + 32 * u;
+        expand_row<DQ>(sK + st * C::kKBytes, cb[u], t * BN + r < N, r, d);
       }
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[kKvFull + s]);
+      if (lane == 0) mbar_arrive(&bars[Bar::kvfull(st)]);
     }
-    // Leave no TMA copy in flight: wait (bounded, even after an abort) for the last two
-    // stages this warp filled.
-    for (int t = (issued > 2 ? issued - 2 : 0); t < issued; ++t)
-      wait_bounded(&bars[kKvFull + (t & 1)], (t >> 1) & 1, abort_flag, false);
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
@@ -247,45 +346,49 @@ __global__ void __launch_bounds__(Cfg<DP>::kThreads, 1)
                                 (static_cast<uint32_t>(BM >> 4) << 24);
       const uint32_t idesc_pv = (2u << 4) | (0u << 7) | (1u << 10) | (1u << 16) |
                                 (static_cast<uint32_t>(DP >> 3) << 17) | (static_cast<uint32_t>(BM >> 4) << 24);
-      if (wait_bounded(&bars[kQFull], 0, abort_flag)) {
+      if (wait_bounded(&bars[Bar::qfull()], 0, abort_flag)) {
         tc_fence_after();
-        for (int t = 0; t <= T; ++t) {
-          if (t < T) {
-            if (!wait_bounded(&bars[kKvFull + (t & 1)], (t >> 1) & 1, abort_flag)) break;
-            tc_fence_after();
-          }
-          bool ok = true;
-          for (int q = 0; q < NQ; ++q) {
+        bool ok = true;
+        for (int t = 0; t <= T && ok; ++t) {
+          for (int q = 0; q < NQ && ok; ++q) {
+            // P.V of the previous block first (it needs no new operands), then QK of this
+            // block into the same S columns (issue order keeps P read before S is rewritten).
             if (t > 0) {
-              if (!wait_bounded(&bars[Bars<NQ>::pfull(q)], (t - 1) & 1, abort_flag)) {
+              if (!wait_bounded(&bars[Bar::pfull(q)], (t - 1) & 1, abort_flag)) {
                 ok = false;
                 break;
               }
               tc_fence_after();
-              const uint32_t vbase = smem_u32(sV + ((t - 1) & 1) * C::kVBytes);
+              const uint32_t vbase = smem_u32(sV + ((t - 1) % S) * C::kVBytes);
 #pragma unroll
               for (int kk = 0; kk < BN / 32; ++kk)
                 mma_i8_ts(tmem + C::tO(q), tmem + C::tP(q) + 8 * kk, smem_desc(vbase + 512 * kk, 128, 2048),
                           idesc_pv, (t > 1 || kk > 0) ? 1u : 0u);
             }
             if (t < T) {
-              const uint32_t qb = smem_u32(sQ + q * C::kQBytes), kb = smem_u32(sK + (t & 1) * C::kKBytes);
+              if (q == 0) {
+                if (!wait_bounded(&bars[Bar::kvfull(t % S)], (t / S) & 1, abort_flag)) {
+                  ok = false;
+                  break;
+                }
+                tc_fence_after();
+              }
+              const uint32_t qb = smem_u32(sQ + q * C::kQBytes), kb = smem_u32(sK + (t % S) * C::kKBytes);
 #pragma unroll
               for (int kk = 0; kk < DQ / 32; ++kk)
                 mma_f8f6f4_ss(tmem + C::tS(q), smem_desc(qb + kk * 4096, 2048, 128),
                               smem_desc(kb + kk * 4096, 2048, 128), idesc_qk, kk > 0 ? 1u : 0u);
-              tc_commit(&bars[kSFull + q]);
+              tc_commit(&bars[Bar::sfull(q)]);
             } else {
-              tc_commit(&bars[Bars<NQ>::odone(q)]);
+              tc_commit(&bars[Bar::odone(q)]);
             }
           }
-          if (!ok) break;
-          if (t > 0) tc_commit(&bars[kKvEmpty + ((t - 1) & 1)]);
+          if (ok && t > 0) tc_commit(&bars[Bar::kvempty((t - 1) % S)]);
         }
       }
       // Every MMA this thread issued has completed before tensor memory is released.
-      tc_commit(&bars[kDrain]);
-      wait_bounded(&bars[kDrain], 0, abort_flag, false);
+      tc_commit(&bars[Bar::drain()]);
+      wait_bounded(&bars[Bar::drain()], 0, abort_flag, false);
     }
     __syncwarp();
   } else if (warp >= 4) {
@@ -299,203 +402,199 @@ __global__ void __launch_bounds__(Cfg<DP>::kThreads, 1)
     const uint32_t aS = tmem + lane_base + C::tS(q);
     const uint32_t aP = tmem + lane_base + C::tP(q);
     const uint32_t aO = tmem + lane_base + C::tO(q);
+    const uint32_t aF = tmem + lane_base + C::tF(q);
     const float alpha = __fmul_rn(__fmul_rn(p.softmax_scale, p.mu_q[bh]), p.mu_k[bh]);
     const float2 alpha2 = make_float2(alpha, alpha);
 
-    // Bias addressing. Dense: this row of [H][N][N]. Rel-pos: b_ij = tab[a_i - koff_j], where
-    // tab is the head's table (in shared memory when staged, followed by zeros that prefix
-    // rows and prefix keys index into).
+    // Bias addressing. Dense: this row of [H][N][N]. Rel-pos: b_ij = tab[a_i - koff_j] with
+    // tab the head's table (staged in shared memory when it fits, followed by zeros that
+    // class-token rows and keys index into), koff_j kept as byte offsets.
     const float* brow = nullptr;
-    const float* tab = nullptr;
+    const float* gtab = nullptr;
     int a_i = 0;
     if (BK == BA_BIAS_DENSE) brow = p.bias.data + b * p.bias.batch_stride + (h * N + ic) * N;
-    if (BK == BA_BIAS_RELPOS2D) {
+    if (is_relpos(BK)) {
       const int W2 = 2 * p.bias.table_w - 1;
-      tab = (tab_mode != 0) ? stab : p.bias.data + h * static_cast<int64_t>(2 * p.bias.table_h - 1) * W2;
+      gtab = p.bias.data + h * static_cast<int64_t>(2 * p.bias.table_h - 1) * W2;
       if (ic >= p.bias.n_prefix) {
         const int ti = ic - p.bias.n_prefix;
         const int yi = ti / p.bias.grid_w;
         a_i = (yi + p.bias.table_h - 1) * W2 + (ti - yi * p.bias.grid_w) + p.bias.table_w - 1;
       } else {
-        a_i = (tab_mode == 2) ? tsize + kmax : -1;  // prefix row: zeros (or the slow path)
+        a_i = (tab_mode == 2) ? tsize + kmax : -1;  // class-token row: the zeros (or the general path)
       }
     }
-    // Fast path: full key blocks, no debug output, aligned dense rows, prefix handled by zeros.
+    const uint32_t tb = smem_u32(stab) + 4u * static_cast<uint32_t>(a_i);  // this row's table base
+    // Fast path: full key blocks, no debug output, aligned dense rows, rel-pos table in shared
+    // memory with the class tokens handled by the zero padding.
     const bool fast_ok = (p.dbg_logits == nullptr) &&
                          (BK != BA_BIAS_DENSE || ((N & 3) == 0 && (p.bias.batch_stride & 3) == 0)) &&
-                         (BK != BA_BIAS_RELPOS2D || p.bias.n_prefix == 0 || tab_mode == 2);
+                         (!is_relpos(BK) || p.bias.n_prefix == 0 || tab_mode == 2);
+    const float* grow = gtab + a_i;  // this row's base in a table left in global memory
 
     float m = -CUDART_INF_F, l = 0.0f;
-    float of[DP];
-#pragma unroll
-    for (int c = 0; c < DP; ++c) of[c] = 0.0f;
     bool alive = true;
 
     for (int t = 0; t < T && alive; ++t) {
-      const int s = t & 1;
+      const int st = t % S;
       const int nk = min(BN, N - t * BN);
-      if (BK == BA_BIAS_RELPOS2D && !wait_warp(&bars[kKvFull + s], (t >> 1) & 1, abort_flag)) {
+      if (is_relpos(BK) && !wait_warp(&bars[Bar::kvfull(st)], (t / S) & 1, abort_flag)) {
         alive = false;
         break;
       }
-      if (!wait_warp(&bars[kSFull + q], t & 1, abort_flag)) {
+      if (!wait_warp(&bars[Bar::sfull(q)], t & 1, abort_flag)) {
         alive = false;
         break;
       }
       tc_fence_after();
-      const int* ko = koff + s * BN;
+      const uint32_t ko_s = smem_u32(koff + st * BN);
 
-      // Pass 1: s = alpha * x + b written back over S in TMEM; block max.
-      float mx0 = -CUDART_INF_F, mx1 = -CUDART_INF_F;
-      if (fast_ok && nk == BN) {
-#pragma unroll 1
+      // Pass 1: s = alpha * x + b written back over S in TMEM; block max. The next 32-column
+      // block is loaded from TMEM while this one is computed.
+      float mx[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
+      // The fast path also takes a partial last block (keys past N are masked to -inf after
+      // the fact; their rel-pos offsets point at valid entries), except for dense bias rows,
+      // which end at N.
+      const bool fast = fast_ok && (nk == BN || BK != BA_BIAS_DENSE);
+      {
+        uint32_t xa[32], xb[32];
+        tmem_ld32(aS, xa);
+#pragma unroll
         for (int c = 0; c < BN / 32; ++c) {
-          float bv[32];
-          if (BK == BA_BIAS_DENSE) {
-            const float4* src = reinterpret_cast<const float4*>(brow + t * BN + 32 * c);
-#pragma unroll
-            for (int k4 = 0; k4 < 8; ++k4) {
-              const float4 v4 = __ldg(src + k4);
-              bv[4 * k4] = v4.x; bv[4 * k4 + 1] = v4.y; bv[4 * k4 + 2] = v4.z; bv[4 * k4 + 3] = v4.w;
-            }
-          } else if (BK == BA_BIAS_RELPOS2D) {
-            const int4* kv = reinterpret_cast<const int4*>(ko + 32 * c);
-#pragma unroll
-            for (int k4 = 0; k4 < 8; ++k4) {
-              const int4 o4 = kv[k4];
-              bv[4 * k4] = tab[a_i - o4.x];
-              bv[4 * k4 + 1] = tab[a_i - o4.y];
-              bv[4 * k4 + 2] = tab[a_i - o4.z];
-              bv[4 * k4 + 3] = tab[a_i - o4.w];
-            }
-          } else {
-#pragma unroll
-            for (int u = 0; u < 32; ++u) bv[u] = 0.0f;
-          }
-          uint32_t x[32];
-          tmem_ld32(aS + 32 * c, x);
-          tmem_ld_wait32(x);
-#pragma unroll
-          for (int k = 0; k < 16; ++k) {
-            const float2 s2 = __ffma2_rn(alpha2, make_float2(__uint_as_float(x[2 * k]), __uint_as_float(x[2 * k + 1])),
-                                         make_float2(bv[2 * k], bv[2 * k + 1]));
-            x[2 * k] = __float_as_uint(s2.x);
-            x[2 * k + 1] = __float_as_uint(s2.y);
-            if (k & 1)
-              mx1 = fmax3(mx1, s2.x, s2.y);
+          uint32_t(&x)[32] = (c & 1) ? xb : xa;
+          uint32_t(&xn)[32] = (c & 1) ? xa : xb;
+          tmem_ld_wait();
+          reg_fence32(x);
+          if (c + 1 < BN / 32) tmem_ld32(aS + 32 * (c + 1), xn);
+          if (fast) {
+            if (nk == BN)
+              fast_block<BK, false>(x, c, nk, alpha2, brow + t * BN, ko_s, tb, grow, tab_mode, mx);
             else
-              mx0 = fmax3(mx0, s2.x, s2.y);
-          }
-          tmem_st32(aS + 32 * c, x);
-        }
-      } else {
-        // General path: a partial last block, prefix tokens without zero padding, unaligned
-        // dense rows, or the debug logits.
-        auto bias_of = [&](int j) -> float {
-          if (BK == BA_BIAS_DENSE) return __ldg(brow + t * BN + j);
-          if (BK == BA_BIAS_RELPOS2D) {
-            const int kj = ko[j];
-            return (a_i >= 0 && kj >= 0) ? tab[a_i - kj] : 0.0f;
-          }
-          return 0.0f;
-        };
-#pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          uint32_t x[32];
-          tmem_ld32(aS + 32 * c, x);
-          tmem_ld_wait32(x);
+              fast_block<BK, true>(x, c, nk, alpha2, brow + t * BN, ko_s, tb, grow, tab_mode, mx);
+          } else {
+            // General path: a partial last block, class tokens without zero padding,
+            // unaligned dense rows, a table in global memory, or the debug logits.
 #pragma unroll
-          for (int u = 0; u < 32; ++u) {
-            const int j = 32 * c + u;
-            float sv = -CUDART_INF_F;
-            if (j < nk) {
-              const float xf = __uint_as_float(x[u]);
-              sv = __fmaf_rn(alpha, xf, bias_of(j));
-              if (p.dbg_logits != nullptr && row_ok)
-                p.dbg_logits[(bh * N + i) * N + t * BN + j] = __float2int_rn(xf);
+            for (int u = 0; u < 32; ++u) {
+              const int j = 32 * c + u;
+              float sv = -CUDART_INF_F;
+              if (j < nk) {
+                const float xf = __uint_as_float(x[u]);
+                float bias = 0.0f;
+                if (BK == BA_BIAS_DENSE) bias = __ldg(brow + t * BN + j);
+                if (is_relpos(BK)) {
+                  const int kj = lds_s32(ko_s + 4u * j) >> 2;
+                  if (a_i >= 0 && kj >= 0)
+                    bias = (tab_mode != 0) ? lds_f32(smem_u32(stab) + 4u * static_cast<uint32_t>(a_i - kj))
+                                           : __ldg(gtab + (a_i - kj));
+                }
+                sv = __fmaf_rn(alpha, xf, bias);
+                if (p.dbg_logits != nullptr && row_ok)
+                  p.dbg_logits[(bh * N + i) * N + t * BN + j] = __float2int_rn(xf);
+              }
+              mx[u & 3] = fmaxf(mx[u & 3], sv);
+              x[u] = __float_as_uint(sv);
             }
-            mx0 = fmaxf(mx0, sv);
-            x[u] = __float_as_uint(sv);
           }
           tmem_st32(aS + 32 * c, x);
         }
       }
-      const float m_new = fmaxf(m, fmaxf(mx0, mx1));
+      const float m_new = fmaxf(m, fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])));
       tmem_st_wait();
 
-      // Pass 2: P~ = 2^((s - m) log2 e) (masked keys hold s = -inf: P~ = 0), row sum, codes -> TMEM.
+      // Pass 2: P~ = 2^((s - m) log2 e) (masked keys hold s = -inf: P~ = 0), row sum, u8 codes
+      // -> TMEM columns 0..31 (their s values were read in the first step of this pass).
       const float2 negm2 = make_float2(-m_new, -m_new);
       const float2 log2e2 = make_float2(kLog2e, kLog2e);
       const float2 c255 = make_float2(255.0f, 255.0f);
       const float2 magic2 = make_float2(12582912.0f, 12582912.0f);
-      float2 lt2 = make_float2(0.0f, 0.0f);
-#pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t x[32];
-        tmem_ld32(aS + 32 * c, x);
-        tmem_ld_wait32(x);
-        uint32_t pk[8];
+      float2 lt2[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
+      {
+        uint32_t xa[32], xb[32];
+        tmem_ld32(aS, xa);
 #pragma unroll
-        for (int w = 0; w < 8; ++w) {
-          uint32_t y[4];
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t(&x)[32] = (c & 1) ? xb : xa;
+          uint32_t(&xn)[32] = (c & 1) ? xa : xb;
+          tmem_ld_wait();
+          reg_fence32(x);
+          if (c + 1 < BN / 32) tmem_ld32(aS + 32 * (c + 1), xn);
+          uint32_t pk[8];
 #pragma unroll
-          for (int e2 = 0; e2 < 2; ++e2) {
-            const int u = 4 * w + 2 * e2;
-            // s - m first (exact near the max), then the scale to base 2.
-            const float2 t2 = __fmul2_rn(
-                __fadd2_rn(make_float2(__uint_as_float(x[u]), __uint_as_float(x[u + 1])), negm2), log2e2);
-            const float2 p2 = make_float2(ex2_approx(t2.x), ex2_approx(t2.y));
-            lt2 = __fadd2_rn(lt2, p2);
-            // 255 P~ + 1.5 * 2^23: one rounding to the nearest integer (ties to even); the
-            // integer sits in the low byte of the result (P~ <= 1).
-            const float2 y2 = __ffma2_rn(p2, c255, magic2);
-            y[2 * e2] = __float_as_uint(y2.x);
-            y[2 * e2 + 1] = __float_as_uint(y2.y);
+          for (int w = 0; w < 8; ++w) {
+            uint32_t y[4];
+#pragma unroll
+            for (int e2 = 0; e2 < 2; ++e2) {
+              const int u = 4 * w + 2 * e2;
+              // s - m first (exact near the max), then the scale to base 2.
+              const float2 t2 = __fmul2_rn(
+                  __fadd2_rn(make_float2(__uint_as_float(x[u]), __uint_as_float(x[u + 1])), negm2), log2e2);
+              const float2 p2 = make_float2(ex2_approx(t2.x), ex2_approx(t2.y));
+              lt2[e2] = __fadd2_rn(lt2[e2], p2);
+              // 255 P~ + 1.5 * 2^23: one rounding to the nearest integer (ties to even); the
+              // integer sits in the low byte of the result (P~ <= 1).
+              const float2 y2 = __ffma2_rn(p2, c255, magic2);
+              y[2 * e2] = __float_as_uint(y2.x);
+              y[2 * e2 + 1] = __float_as_uint(y2.y);
+            }
+            pk[w] = __byte_perm(__byte_perm(y[0], y[1], 0x0040), __byte_perm(y[2], y[3], 0x0040), 0x5410);
           }
-          pk[w] = __byte_perm(__byte_perm(y[0], y[1], 0x0040), __byte_perm(y[2], y[3], 0x0040), 0x5410);
+          tmem_st8(aP + 8 * c, pk);
         }
-        tmem_st8(aP + 8 * c, pk);
       }
-      const float lt = lt2.x + lt2.y;
+      const float lt = (lt2[0].x + lt2[0].y) + (lt2[1].x + lt2[1].y);
       const float ct = (m == -CUDART_INF_F) ? 0.0f : ex2_approx((m - m_new) * kLog2e);
       l = l * ct + lt;
+      // Fold the int32 accumulator into the fp32 running output F when the row max rose
+      // (t = 0: F starts at zero and P.V overwrites the accumulator).
       const bool flush = (t > 0) && (m_new > m);
-      if (__any_sync(0xffffffffu, flush)) {
+      if (t == 0 || __any_sync(0xffffffffu, flush)) {
 #pragma unroll
         for (int cc = 0; cc < DP / 16; ++cc) {
-          uint32_t a[16];
-          tmem_ld16(aO + 16 * cc, a);
-          tmem_ld_wait16(a);
-          if (flush) {
+          uint32_t a[16], f[16];
+          if (t > 0) {
+            tmem_ld16(aO + 16 * cc, a);
+            tmem_ld16(aF + 16 * cc, f);
+            tmem_ld_wait();
+            reg_fence16(a);
+            reg_fence16(f);
+          }
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              of[16 * cc + e] = (of[16 * cc + e] + __int2float_rn(static_cast<int>(a[e]))) * ct;
+          for (int e = 0; e < 16; ++e) {
+            if (t == 0) {
+              f[e] = 0u;
+            } else if (flush) {
+              f[e] = __float_as_uint((__uint_as_float(f[e]) + __int2float_rn(static_cast<int>(a[e]))) * ct);
               a[e] = 0u;
             }
           }
-          tmem_st16(aO + 16 * cc, a);
+          if (t > 0) tmem_st16(aO + 16 * cc, a);
+          tmem_st16(aF + 16 * cc, f);
         }
       }
       m = m_new;
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[Bars<NQ>::pfull(q)]);
+      if (lane == 0) mbar_arrive(&bars[Bar::pfull(q)]);
     }
 
-    if (alive && wait_warp(&bars[Bars<NQ>::odone(q)], 0, abort_flag)) {
+    if (alive && wait_warp(&bars[Bar::odone(q)], 0, abort_flag)) {
       tc_fence_after();
       const float inv_l = 1.0f / l;
 #pragma unroll
       for (int cc = 0; cc < DP / 16; ++cc) {
-        uint32_t a[16];
+        uint32_t a[16], f[16];
         tmem_ld16(aO + 16 * cc, a);
-        tmem_ld_wait16(a);
+        tmem_ld16(aF + 16 * cc, f);
+        tmem_ld_wait();
+        reg_fence16(a);
+        reg_fence16(f);
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           const int c = 16 * cc + e;
           if (row_ok && c < d) {
-            const float val = (of[c] + __int2float_rn(static_cast<int>(a[e]))) * sscale[c] * inv_l;
+            const float val = (__uint_as_float(f[e]) + __int2float_rn(static_cast<int>(a[e]))) * sscale[c] * inv_l;
             store_out(p.o, (bh * N + i) * d + c, val, p.o_dt);
           }
         }
@@ -504,13 +603,11 @@ __global__ void __launch_bounds__(Cfg<DP>::kThreads, 1)
   }
 
   // ------------------------------------------------------------ teardown
-  if (warp != 2 && warp != 3) {
-    tc_fence_before();
-    named_barrier_sync(1, C::kThreads - 64);
-    if (warp == 1) {
-      tc_fence_after();
-      tmem_dealloc(tmem, 512);
-    }
+  tc_fence_before();
+  named_barrier_sync(1, C::kThreads);
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
   }
 }
 
@@ -533,18 +630,25 @@ EncodeTiledFn encode_fn() {
 
 constexpr int kMaxSmem = 227 * 1024;
 
+// 0: rel-pos table read from global memory; 1: staged in shared memory; 2: staged and followed
+// by 2 * tsize zeros that class-token rows and keys index into.
+template <int DP>
+int relpos_table_mode(const AttnParams& p) {
+  const int64_t tsize = static_cast<int64_t>(2 * p.bias.table_h - 1) * (2 * p.bias.table_w - 1);
+  const int64_t room = kMaxSmem - 1024 - Cfg<DP>::kTabOff;
+  if (p.bias.n_prefix > 0 && 3 * tsize * 4 <= room) return 2;
+  if (tsize * 4 <= room) return 1;
+  return 0;
+}
+
 template <int DP, int BK>
 cudaError_t launch_dp_bk(const AttnParams& p, const CUtensorMap& tm, cudaStream_t s) {
   using C = Cfg<DP>;
   int tab_mode = 0, tsize = 0, kmax = 0;
-  if (BK == BA_BIAS_RELPOS2D) {
+  if (is_relpos(BK)) {
     tsize = (2 * p.bias.table_h - 1) * (2 * p.bias.table_w - 1);
     kmax = (p.bias.grid_h - 1) * (2 * p.bias.table_w - 1) + p.bias.grid_w - 1;
-    const int64_t room = kMaxSmem - 1024 - C::kTabOff;
-    if (p.bias.n_prefix > 0 && 3ll * tsize * 4 <= room)
-      tab_mode = 2;
-    else if (static_cast<int64_t>(tsize) * 4 <= room)
-      tab_mode = 1;
+    tab_mode = relpos_table_mode<DP>(p);
   }
   const int tab_bytes = tab_mode == 0 ? 0 : (tab_mode == 2 ? 3 : 1) * tsize * 4;
   // At least 116 KB of shared memory per CTA keeps one CTA per SM (it owns all 512 TMEM columns).
@@ -565,7 +669,9 @@ template <int DP>
 cudaError_t launch_dp(const AttnParams& p, const CUtensorMap& tm, cudaStream_t s) {
   switch (p.bias.kind) {
     case BA_BIAS_DENSE: return launch_dp_bk<DP, BA_BIAS_DENSE>(p, tm, s);
-    case BA_BIAS_RELPOS2D: return launch_dp_bk<DP, BA_BIAS_RELPOS2D>(p, tm, s);
+    case BA_BIAS_RELPOS2D:
+      return relpos_table_mode<DP>(p) != 0 ? launch_dp_bk<DP, BA_BIAS_RELPOS2D>(p, tm, s)
+                                           : launch_dp_bk<DP, kRelposGlobal>(p, tm, s);
     default: return launch_dp_bk<DP, BA_BIAS_NONE>(p, tm, s);
   }
 }
