@@ -582,6 +582,11 @@ __global__ void __launch_bounds__(Cfg<DP>::kThreads, 1)
     if (alive && wait_warp(&bars[Bar::odone(q)], 0, abort_flag)) {
       tc_fence_after();
       const float inv_l = 1.0f / l;
+      // Rows whose byte length is a multiple of 16 are written with 16-byte stores (each
+      // thread owns one row); other shapes fall back to element stores.
+      const int esz = (p.o_dt == BA_F32) ? 4 : 2;
+      const bool vec = ((d * esz) & 15) == 0;
+      char* orow = reinterpret_cast<char*>(p.o) + ((bh * N + i) * d) * esz;
 #pragma unroll
       for (int cc = 0; cc < DP / 16; ++cc) {
         uint32_t a[16], f[16];
@@ -590,13 +595,36 @@ __global__ void __launch_bounds__(Cfg<DP>::kThreads, 1)
         tmem_ld_wait();
         reg_fence16(a);
         reg_fence16(f);
+        float val[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int c = 16 * cc + e;
-          if (row_ok && c < d) {
-            const float val = (__uint_as_float(f[e]) + __int2float_rn(static_cast<int>(a[e]))) * sscale[c] * inv_l;
-            store_out(p.o, (bh * N + i) * d + c, val, p.o_dt);
+        for (int e = 0; e < 16; ++e)
+          val[e] = (__uint_as_float(f[e]) + __int2float_rn(static_cast<int>(a[e]))) * sscale[16 * cc + e] * inv_l;
+        if (!row_ok) continue;
+        if (vec && 16 * cc + 16 <= d) {
+          if (p.o_dt == BA_F32) {
+#pragma unroll
+            for (int k4 = 0; k4 < 4; ++k4)
+              reinterpret_cast<float4*>(orow + (16 * cc + 4 * k4) * 4)[0] =
+                  make_float4(val[4 * k4], val[4 * k4 + 1], val[4 * k4 + 2], val[4 * k4 + 3]);
+          } else {
+            uint32_t h[8];
+#pragma unroll
+            for (int k2 = 0; k2 < 8; ++k2) {
+              if (p.o_dt == BA_F16) {
+                const __half2 v = __floats2half2_rn(val[2 * k2], val[2 * k2 + 1]);
+                h[k2] = *reinterpret_cast<const uint32_t*>(&v);
+              } else {
+                const __nv_bfloat162 v = __floats2bfloat162_rn(val[2 * k2], val[2 * k2 + 1]);
+                h[k2] = *reinterpret_cast<const uint32_t*>(&v);
+              }
+            }
+            reinterpret_cast<uint4*>(orow + 16 * cc * 2)[0] = make_uint4(h[0], h[1], h[2], h[3]);
+            reinterpret_cast<uint4*>(orow + 16 * cc * 2)[1] = make_uint4(h[4], h[5], h[6], h[7]);
           }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            if (16 * cc + e < d) store_out(p.o, (bh * N + i) * d + 16 * cc + e, val[e], p.o_dt);
         }
       }
     }
