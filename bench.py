@@ -35,10 +35,11 @@ KERNEL_FILES = {"stream_qkv": "prep.cu", "finalize": "prep.cu", "quant_v": "prep
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--steps", type=int, default=6000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="deit_b")
+    ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (small profiling cases)")
     ap.add_argument("--attn-impl", choices=["auto", "simt", "tcgen05"], default="auto")
     ap.add_argument("--rotate", type=int, default=0, help="input sets cycled to defeat L2 (0 = auto)")
     ap.add_argument("--e2e-steps", type=int, default=20)
@@ -93,7 +94,7 @@ class ClockSampler:
             os.close(fd)
             self.out = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
                                          stdout=self.out, stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
@@ -225,6 +226,10 @@ def main():
     ba.set_attention_impl({"auto": 0, "simt": 1, "tcgen05": 2}[args.attn_impl])
 
     w = inputs.by_name(args.workload)
+    if args.batch:
+        w.B = args.batch
+        w.q, w.k, w.v = (t[:args.batch].contiguous() for t in (w.q, w.k, w.v))
+        w.name = f"{w.name}[B={args.batch}]"
     ops, tokens = work_units(w)
     E = w.B * w.H * w.N * w.d
     esz = 2
