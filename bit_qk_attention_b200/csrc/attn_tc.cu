@@ -457,15 +457,14 @@ __global__ void __launch_bounds__(Cfg<DP>::kThreads, 1)
       // which end at N.
       const bool fast = fast_ok && (nk == BN || BK != BA_BIAS_DENSE);
       {
-        uint32_t xa[32], xb[32];
-        tmem_ld32(aS, xa);
-#pragma unroll
+        // One copy of the block body (a small hot loop stays in the instruction cache; the
+        // other softmax warps of the SM cover the TMEM load latency).
+#pragma unroll 1
         for (int c = 0; c < BN / 32; ++c) {
-          uint32_t(&x)[32] = (c & 1) ? xb : xa;
-          uint32_t(&xn)[32] = (c & 1) ? xa : xb;
+          uint32_t x[32];
+          tmem_ld32(aS + 32 * c, x);
           tmem_ld_wait();
           reg_fence32(x);
-          if (c + 1 < BN / 32) tmem_ld32(aS + 32 * (c + 1), xn);
           if (fast) {
             if (nk == BN)
               fast_block<BK, false>(x, c, nk, alpha2, brow + t * BN, ko_s, tb, grow, tab_mode, mx);
@@ -510,15 +509,12 @@ __global__ void __launch_bounds__(Cfg<DP>::kThreads, 1)
       const float2 magic2 = make_float2(12582912.0f, 12582912.0f);
       float2 lt2[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
       {
-        uint32_t xa[32], xb[32];
-        tmem_ld32(aS, xa);
-#pragma unroll
+#pragma unroll 1
         for (int c = 0; c < BN / 32; ++c) {
-          uint32_t(&x)[32] = (c & 1) ? xb : xa;
-          uint32_t(&xn)[32] = (c & 1) ? xa : xb;
+          uint32_t x[32];
+          tmem_ld32(aS + 32 * c, x);
           tmem_ld_wait();
           reg_fence32(x);
-          if (c + 1 < BN / 32) tmem_ld32(aS + 32 * (c + 1), xn);
           uint32_t pk[8];
 #pragma unroll
           for (int w = 0; w < 8; ++w) {
@@ -549,7 +545,7 @@ __global__ void __launch_bounds__(Cfg<DP>::kThreads, 1)
       // (t = 0: F starts at zero and P.V overwrites the accumulator).
       const bool flush = (t > 0) && (m_new > m);
       if (t == 0 || __any_sync(0xffffffffu, flush)) {
-#pragma unroll
+#pragma unroll 1
         for (int cc = 0; cc < DP / 16; ++cc) {
           uint32_t a[16], f[16];
           if (t > 0) {
