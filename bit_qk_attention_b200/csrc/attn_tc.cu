@@ -7,10 +7,13 @@
 // on every page).
 //
 // How, on B200:
-//   * One CTA per SM; each CTA owns NQ query tiles of 128 rows of one (b, h).
-//   * Warp 0 (producer) expands the 1-bit sign rows of Q (once) and of each K block into fp8
-//     +-1 operands in shared memory (channels >= d become 0), and TMA-loads the int8 V block
-//     (a 4-D tensor map that lands it in the MN-major core-matrix layout the MMA reads).
+//   * Each CTA owns NQ query tiles of 128 rows of one (b, h): one tile in 256 tensor-memory
+//     columns (two CTAs per SM) when the head and the bias table fit, else two tiles in 512.
+//   * Warps 2 and 3 expand the 1-bit sign rows of Q (once) and of each K block into fp8 +-1
+//     operands in shared memory (channels >= d become 0); warp 0 TMA-loads the int8 V block
+//     (a 4-D tensor map that lands it in the MN-major core-matrix layout the MMA reads) and
+//     writes the block's rel-pos key offsets. A 4-stage ring of K/V blocks decouples them from
+//     the MMAs.
 //   * Warp 1 issues the MMAs from one thread:
 //       S  = Q . K^T   tcgen05.mma kind::f8f6f4 (e4m3 +-1, fp32 accumulate: exact integers)
 //       O += P . V     tcgen05.mma kind::i8, A = the uint8 codes read from TMEM, B = int8 V
@@ -46,10 +49,10 @@ constexpr int BN = kKvBlock;   // keys per block = MMA N of QK, K of P.V
 constexpr uint64_t kTimeoutNs = 1000000000ull;
 constexpr float kLog2e = 1.4426950408889634f;
 
-template <int DP>
+template <int DP, int NQ_>
 struct Cfg {
   static constexpr int DQ = (DP + 31) / 32 * 32;   // QK contraction width: fp8 K-steps of 32
-  static constexpr int NQ = (DP <= 64) ? 2 : 1;     // query tiles per CTA
+  static constexpr int NQ = NQ_;                    // query tiles per CTA
   static constexpr int kThreads = 128 + 128 * NQ;   // 4 service warps + NQ softmax warpgroups
   static constexpr int kQBytes = BM * DQ;
   static constexpr int kKBytes = BN * DQ;
@@ -74,6 +77,10 @@ struct Cfg {
   __host__ __device__ static constexpr uint32_t tO(int q) { return q * 256 + 128; }
   __host__ __device__ static constexpr uint32_t tF(int q) { return q * 256 + 128 + DP; }
   static_assert(tF(NQ - 1) + DP <= 512, "tensor memory budget");
+  // Columns allocated: a CTA whose tiles fit in half of tensor memory takes 256 columns and
+  // shares its SM with a second CTA.
+  static constexpr int kTmemCols = (tF(NQ - 1) + DP <= 256) ? 256 : 512;
+  static constexpr int kCtasPerSm = 512 / kTmemCols;
 };
 
 // Barrier slots: kv_full[S], kv_empty[S], q_full, drain, s_full[NQ], p_full[NQ], o_done[NQ].
@@ -191,11 +198,11 @@ __device__ __forceinline__ void fast_block(uint32_t (&x)[32], int c, int nk, flo
   }
 }
 
-template <int DP, int BK>
-__global__ void __launch_bounds__(Cfg<DP>::kThreads, 1)
+template <int DP, int BK, int NQ_>
+__global__ void __launch_bounds__(Cfg<DP, NQ_>::kThreads, Cfg<DP, NQ_>::kCtasPerSm)
     attn_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmap_v, int tab_mode, int tsize,
                    int kmax) {
-  using C = Cfg<DP>;
+  using C = Cfg<DP, NQ_>;
   constexpr int NQ = C::NQ, DQ = C::DQ, S = C::kStages;
   using Bar = Bars<S, NQ>;
   extern __shared__ uint8_t smem_raw[];
@@ -246,7 +253,7 @@ __global__ void __launch_bounds__(Cfg<DP>::kThreads, 1)
     for (int e = threadIdx.x; e < n; e += C::kThreads) stab[e] = (e < tsize) ? __ldg(src + e) : 0.0f;
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, 512);
+    tmem_alloc(tmem_slot, C::kTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -438,6 +445,9 @@ __global__ void __launch_bounds__(Cfg<DP>::kThreads, 1)
     for (int t = 0; t < T && alive; ++t) {
       const int st = t % S;
       const int nk = min(BN, N - t * BN);
+      // 32-key chunks that hold keys of this block. The P codes of the chunks past them are
+      // left as they are: they multiply V rows past N, which the V copy fills with zeros.
+      const int nch = (nk + 31) >> 5;
       if (is_relpos(BK) && !wait_warp(&bars[Bar::kvfull(st)], (t / S) & 1, abort_flag)) {
         alive = false;
         break;
@@ -460,7 +470,7 @@ __global__ void __launch_bounds__(Cfg<DP>::kThreads, 1)
         // One copy of the block body (a small hot loop stays in the instruction cache; the
         // other softmax warps of the SM cover the TMEM load latency).
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
+        for (int c = 0; c < nch; ++c) {
           uint32_t x[32];
           tmem_ld32(aS + 32 * c, x);
           tmem_ld_wait();
@@ -510,7 +520,7 @@ __global__ void __launch_bounds__(Cfg<DP>::kThreads, 1)
       float2 lt2[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
       {
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
+        for (int c = 0; c < nch; ++c) {
           uint32_t x[32];
           tmem_ld32(aS + 32 * c, x);
           tmem_ld_wait();
@@ -631,7 +641,7 @@ __global__ void __launch_bounds__(Cfg<DP>::kThreads, 1)
   named_barrier_sync(1, C::kThreads);
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem, C::kTmemCols);
   }
 }
 
@@ -652,51 +662,75 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-constexpr int kMaxSmem = 227 * 1024;
+constexpr int kMaxSmem = 227 * 1024;      // per CTA
+constexpr int kSmPerSmem = 228 * 1024;    // per SM
+constexpr int kSmemReserved = 1024;       // per CTA, taken by the runtime
+
+// Dynamic shared memory a CTA of configuration C may use.
+template <class C>
+constexpr int smem_room() {
+  return C::kCtasPerSm == 1 ? kMaxSmem : kSmPerSmem / C::kCtasPerSm - kSmemReserved;
+}
 
 // 0: rel-pos table read from global memory; 1: staged in shared memory; 2: staged and followed
 // by 2 * tsize zeros that class-token rows and keys index into.
-template <int DP>
+template <class C>
 int relpos_table_mode(const AttnParams& p) {
   const int64_t tsize = static_cast<int64_t>(2 * p.bias.table_h - 1) * (2 * p.bias.table_w - 1);
-  const int64_t room = kMaxSmem - 1024 - Cfg<DP>::kTabOff;
+  const int64_t room = smem_room<C>() - 1024 - C::kTabOff;
   if (p.bias.n_prefix > 0 && 3 * tsize * 4 <= room) return 2;
   if (tsize * 4 <= room) return 1;
   return 0;
 }
 
-template <int DP, int BK>
-cudaError_t launch_dp_bk(const AttnParams& p, const CUtensorMap& tm, cudaStream_t s) {
-  using C = Cfg<DP>;
+template <int DP, int BK, int NQ>
+cudaError_t launch_cfg(const AttnParams& p, const CUtensorMap& tm, cudaStream_t s) {
+  using C = Cfg<DP, NQ>;
   int tab_mode = 0, tsize = 0, kmax = 0;
   if (is_relpos(BK)) {
     tsize = (2 * p.bias.table_h - 1) * (2 * p.bias.table_w - 1);
     kmax = (p.bias.grid_h - 1) * (2 * p.bias.table_w - 1) + p.bias.grid_w - 1;
-    tab_mode = relpos_table_mode<DP>(p);
+    tab_mode = relpos_table_mode<C>(p);
   }
   const int tab_bytes = tab_mode == 0 ? 0 : (tab_mode == 2 ? 3 : 1) * tsize * 4;
-  // At least 116 KB of shared memory per CTA keeps one CTA per SM (it owns all 512 TMEM columns).
+  // A CTA that owns all 512 tensor-memory columns takes enough shared memory to be alone on its
+  // SM; one that owns 256 takes enough that no third CTA fits.
   int smem = C::kTabOff + tab_bytes + 1024;
-  if (smem < 116 * 1024) smem = 116 * 1024;
+  const int floor_bytes = C::kCtasPerSm == 1 ? 116 * 1024 : 80 * 1024;
+  if (smem < floor_bytes) smem = floor_bytes;
   static int configured = 0;
   if (smem > configured) {
-    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<DP, BK>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<DP, BK, NQ>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     configured = smem;
   }
   const int64_t grid = static_cast<int64_t>(p.B) * p.H * ceil_div(p.N, BM * C::NQ);
-  attn_tc_kernel<DP, BK><<<static_cast<unsigned>(grid), C::kThreads, smem, s>>>(p, tm, tab_mode, tsize, kmax);
+  attn_tc_kernel<DP, BK, NQ><<<static_cast<unsigned>(grid), C::kThreads, smem, s>>>(p, tm, tab_mode, tsize, kmax);
   return cudaGetLastError();
 }
 
+template <int DP, int NQ>
+cudaError_t launch_nq(const AttnParams& p, const CUtensorMap& tm, cudaStream_t s) {
+  switch (p.bias.kind) {
+    case BA_BIAS_DENSE: return launch_cfg<DP, BA_BIAS_DENSE, NQ>(p, tm, s);
+    case BA_BIAS_RELPOS2D:
+      return relpos_table_mode<Cfg<DP, NQ>>(p) != 0 ? launch_cfg<DP, BA_BIAS_RELPOS2D, NQ>(p, tm, s)
+                                                     : launch_cfg<DP, kRelposGlobal, NQ>(p, tm, s);
+    default: return launch_cfg<DP, BA_BIAS_NONE, NQ>(p, tm, s);
+  }
+}
+
+// Head dimensions up to 64 run one query tile per CTA in half of tensor memory, two CTAs per
+// SM (the CTAs' prologues, pipeline fills and epilogues overlap each other's work), unless the
+// rel-pos table only fits in the shared memory of a CTA that has the SM to itself; then one CTA
+// runs two tiles.
 template <int DP>
 cudaError_t launch_dp(const AttnParams& p, const CUtensorMap& tm, cudaStream_t s) {
-  switch (p.bias.kind) {
-    case BA_BIAS_DENSE: return launch_dp_bk<DP, BA_BIAS_DENSE>(p, tm, s);
-    case BA_BIAS_RELPOS2D:
-      return relpos_table_mode<DP>(p) != 0 ? launch_dp_bk<DP, BA_BIAS_RELPOS2D>(p, tm, s)
-                                           : launch_dp_bk<DP, kRelposGlobal>(p, tm, s);
-    default: return launch_dp_bk<DP, BA_BIAS_NONE>(p, tm, s);
+  if constexpr (DP <= 64) {
+    const bool table_fits = p.bias.kind != BA_BIAS_RELPOS2D || relpos_table_mode<Cfg<DP, 1>>(p) != 0;
+    return table_fits ? launch_nq<DP, 1>(p, tm, s) : launch_nq<DP, 2>(p, tm, s);
+  } else {
+    return launch_nq<DP, 1>(p, tm, s);
   }
 }
 
