@@ -21,10 +21,12 @@
 //   * Warpgroup 1+q (one thread per query row) runs the softmax of query tile q: it reads its
 //     row of S from TMEM, forms s = fmaf(alpha, x, b), the running max, P~ = 2^((s-m) log2 e),
 //     the row sum, and writes the 8-bit codes back to TMEM as the A operand of P.V.
-//   * The int32 P.V accumulator keeps accumulating across key blocks while a row's running max
-//     is unchanged (the rescale factor is exactly 1 then); when a row's max rises the thread
-//     folds the accumulator into its fp32 running output, O~ = (O~ + acc) * exp(m_old - m_new),
-//     and zeroes the accumulator row. This is the same arithmetic as rescaling every block.
+//   * The int32 P.V accumulator keeps accumulating across key blocks while no row of the tile
+//     raises its running max (every rescale factor is exactly 1 then). When a row's max rises,
+//     P.V of that block starts the tile's second accumulator instead, and while the MMAs run
+//     the softmax threads fold the first one into their fp32 running outputs,
+//     O~ = (O~ + acc) * exp(m_old - m_new) (factor 1 for rows whose max did not rise). This is
+//     the same arithmetic as rescaling every block, off the softmax's critical path.
 //   * Every wait is bounded (1 s): on expiry the kernel records BA_ERR_TIMEOUT in a device
 //     status word, every role leaves its loop, and the CTA frees its tensor memory.
 #include <cuda.h>
@@ -54,10 +56,13 @@ struct Cfg {
   static constexpr int DQ = (DP + 31) / 32 * 32;   // QK contraction width: fp8 K-steps of 32
   static constexpr int NQ = NQ_;                    // query tiles per CTA
   static constexpr int kThreads = 128 + 128 * NQ;   // 4 service warps + NQ softmax warpgroups
+  // The fp32 running output F of a row lives in shared memory for heads up to 64 wide (tensor
+  // memory then holds S and two accumulators per tile), else in tensor memory.
+  static constexpr bool kFSmem = DP <= 64;
   static constexpr int kQBytes = BM * DQ;
   static constexpr int kKBytes = BN * DQ;
   static constexpr int kVBytes = BN * DP;
-  static constexpr int kStages = 4;                 // K/V pipeline depth
+  static constexpr int kStages = (NQ == 1 && DP <= 64) ? 3 : 4;  // K/V pipeline depth
   static constexpr int offQ = 0;
   static constexpr int offK = offQ + NQ * kQBytes;
   static constexpr int offV = offK + kStages * kKBytes;
@@ -65,21 +70,27 @@ struct Cfg {
   static constexpr int offScale = offKoff + kStages * BN * 4;
   static constexpr int offBar = offScale + 128 * 4;
   static constexpr int kNumBars = 2 * kStages + 2 + 3 * NQ;
-  static constexpr int offMisc = offBar + kNumBars * 8;
-  static constexpr int kBytes = offMisc + 16;
+  static constexpr int offMisc = offBar + kNumBars * 8;           // tmem base, abort flag
+  static constexpr int offVotes = offMisc + 16;                    // [2][NQ][4] u32
+  static constexpr int offF = (offVotes + 2 * NQ * 4 * 4 + 15) / 16 * 16;
+  static constexpr int kFBytes = kFSmem ? NQ * BM * DP * 4 : 0;   // [DP/4][NQ*128] float4
+  static constexpr int kBytes = offF + kFBytes;
   static constexpr int kTabOff = (kBytes + 127) / 128 * 128;
   // Tensor-memory columns of query tile q: S (fp32, 128 columns; the softmax overwrites it
   // with s and then its first 32 columns with the u8 codes P — the MMAs of one CTA run in
-  // issue order, so P.V reads P before the next QK rewrites S), O (the s32 P.V accumulator,
-  // DP) and F (the fp32 running output, DP).
+  // issue order, so P.V reads P before the next QK rewrites S), two s32 P.V accumulators
+  // O0/O1 (DP each: P.V switches to the other one when a row's max rises, while the softmax
+  // threads fold the first into F) and, for wide heads, F (fp32, DP).
   __host__ __device__ static constexpr uint32_t tS(int q) { return q * 256; }
   __host__ __device__ static constexpr uint32_t tP(int q) { return q * 256; }
-  __host__ __device__ static constexpr uint32_t tO(int q) { return q * 256 + 128; }
-  __host__ __device__ static constexpr uint32_t tF(int q) { return q * 256 + 128 + DP; }
-  static_assert(tF(NQ - 1) + DP <= 512, "tensor memory budget");
+  __host__ __device__ static constexpr uint32_t tO(int q, int b) { return q * 256 + 128 + b * DP; }
+  __host__ __device__ static constexpr uint32_t tF(int q) { return q * 256 + 128 + 2 * DP; }
+  static constexpr int kTmemUsed = tO(NQ - 1, 1) + DP + (kFSmem ? 0 : DP);
+  static_assert(kTmemUsed <= 512, "tensor memory budget");
+  static_assert(NQ == 1 || kFSmem, "two tiles per CTA need F in shared memory");
   // Columns allocated: a CTA whose tiles fit in half of tensor memory takes 256 columns and
   // shares its SM with a second CTA.
-  static constexpr int kTmemCols = (tF(NQ - 1) + DP <= 256) ? 256 : 512;
+  static constexpr int kTmemCols = kTmemUsed <= 256 ? 256 : 512;
   static constexpr int kCtasPerSm = 512 / kTmemCols;
 };
 
@@ -198,6 +209,93 @@ __device__ __forceinline__ void fast_block(uint32_t (&x)[32], int c, int nk, flo
   }
 }
 
+// Folding an s32 P.V accumulator row into the fp32 running output of the row:
+// F = (F + acc) * ct, in groups of NC chunks of 16 columns starting at chunk C0. fold_load
+// issues a group's tensor-memory loads (the accumulator, and F when it lives in tensor
+// memory); fold_finish waits for them and completes the group. `fresh`: F holds nothing yet
+// (read as 0). `one_block`: the accumulator holds a single block's P.V,
+// |acc| <= 255 * 127 * 128 < 2^22, which converts exactly by adding it to the bit pattern of
+// 1.5 * 2^23 and subtracting that value as a float; otherwise the hardware conversion is used.
+// F lives in shared memory ([DP/4][NQ*128] float4, `fr` = this row's first entry) or in tensor
+// memory (`aF`).
+template <class C>
+struct FoldShape {
+  static constexpr int NCH = C::kVBytes / BN / 16;  // chunks per row
+  // 2 chunks per group when F is in shared memory (those CTAs share an SM: 128 registers per
+  // thread), 4 when it is in tensor memory.
+  static constexpr int G = C::kFSmem ? 2 : 4;
+  __host__ __device__ static constexpr int nc(int c0) { return (NCH - c0 < G) ? NCH - c0 : G; }
+};
+
+template <class C, int C0, int NC>
+__device__ __forceinline__ void fold_load(uint32_t acc, uint32_t aF, bool fresh, uint32_t (&a)[NC][16],
+                                          uint32_t (&fb)[NC][16]) {
+#pragma unroll
+  for (int k = 0; k < NC; ++k) {
+    tmem_ld16(acc + 16 * (C0 + k), a[k]);
+    if (!C::kFSmem && !fresh) tmem_ld16(aF + 16 * (C0 + k), fb[k]);
+  }
+}
+
+template <class C, int C0, int NC>
+__device__ __forceinline__ void fold_finish(uint32_t aF, float4* fr, float2 ct2, bool fresh, bool one_block,
+                                            uint32_t (&a)[NC][16], uint32_t (&fb)[NC][16]) {
+  tmem_ld_wait();
+#pragma unroll
+  for (int k = 0; k < NC; ++k) {
+    reg_fence16(a[k]);
+    if (!C::kFSmem && !fresh) reg_fence16(fb[k]);
+  }
+#pragma unroll
+  for (int k = 0; k < NC; ++k) {
+    float f[16];
+    if constexpr (C::kFSmem) {
+#pragma unroll
+      for (int k4 = 0; k4 < 4; ++k4) {
+        const float4 v = fresh ? make_float4(0.0f, 0.0f, 0.0f, 0.0f) : fr[(4 * (C0 + k) + k4) * (C::NQ * BM)];
+        f[4 * k4] = v.x; f[4 * k4 + 1] = v.y; f[4 * k4 + 2] = v.z; f[4 * k4 + 3] = v.w;
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 16; ++e) f[e] = fresh ? 0.0f : __uint_as_float(fb[k][e]);
+    }
+#pragma unroll
+    for (int e = 0; e < 16; e += 2) {
+      float2 av;
+      if (one_block) {
+        av = __fadd2_rn(make_float2(__uint_as_float(a[k][e] + 0x4B400000u), __uint_as_float(a[k][e + 1] + 0x4B400000u)),
+                        make_float2(-12582912.0f, -12582912.0f));
+      } else {
+        av = make_float2(__int2float_rn(static_cast<int>(a[k][e])), __int2float_rn(static_cast<int>(a[k][e + 1])));
+      }
+      const float2 v = __fmul2_rn(__fadd2_rn(make_float2(f[e], f[e + 1]), av), ct2);
+      f[e] = v.x; f[e + 1] = v.y;
+    }
+    if constexpr (C::kFSmem) {
+#pragma unroll
+      for (int k4 = 0; k4 < 4; ++k4)
+        fr[(4 * (C0 + k) + k4) * (C::NQ * BM)] = make_float4(f[4 * k4], f[4 * k4 + 1], f[4 * k4 + 2], f[4 * k4 + 3]);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 16; ++e) fb[k][e] = __float_as_uint(f[e]);
+      tmem_st16(aF + 16 * (C0 + k), fb[k]);
+    }
+  }
+}
+
+// The groups from chunk C0 to the end of the row.
+template <class C, int C0>
+__device__ __forceinline__ void fold_rest(uint32_t acc, uint32_t aF, float4* fr, float2 ct2, bool fresh,
+                                          bool one_block) {
+  if constexpr (C0 < FoldShape<C>::NCH) {
+    constexpr int NC = FoldShape<C>::nc(C0);
+    uint32_t a[NC][16], fb[NC][16];
+    fold_load<C, C0, NC>(acc, aF, fresh, a, fb);
+    fold_finish<C, C0, NC>(aF, fr, ct2, fresh, one_block, a, fb);
+    fold_rest<C, C0 + NC>(acc, aF, fr, ct2, fresh, one_block);
+  }
+}
+
 template <int DP, int BK, int NQ_>
 __global__ void __launch_bounds__(Cfg<DP, NQ_>::kThreads, Cfg<DP, NQ_>::kCtasPerSm)
     attn_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmap_v, int tab_mode, int tsize,
@@ -215,6 +313,9 @@ __global__ void __launch_bounds__(Cfg<DP, NQ_>::kThreads, Cfg<DP, NQ_>::kCtasPer
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::offBar);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::offMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::offMisc + 4);
+  // Per block parity, tile and softmax warp: whether a row of that warp raised its max.
+  uint32_t* votes = reinterpret_cast<uint32_t*>(smem + C::offVotes);
+  float4* sF = reinterpret_cast<float4*>(smem + C::offF);  // [DP/4][NQ*128]
   // Rel-pos table of this CTA's head, staged when it fits: tab_mode 1 = table only,
   // 2 = table followed by 2*tsize zeros (targets of prefix rows and prefix keys).
   float* stab = reinterpret_cast<float*>(smem + C::kTabOff);
@@ -356,6 +457,7 @@ __global__ void __launch_bounds__(Cfg<DP, NQ_>::kThreads, Cfg<DP, NQ_>::kCtasPer
       if (wait_bounded(&bars[Bar::qfull()], 0, abort_flag)) {
         tc_fence_after();
         bool ok = true;
+        uint32_t cur_acc = 0;  // bit q: the accumulator P.V of tile q adds into
         for (int t = 0; t <= T && ok; ++t) {
           for (int q = 0; q < NQ && ok; ++q) {
             // P.V of the previous block first (it needs no new operands), then QK of this
@@ -366,11 +468,23 @@ __global__ void __launch_bounds__(Cfg<DP, NQ_>::kThreads, Cfg<DP, NQ_>::kCtasPer
                 break;
               }
               tc_fence_after();
+              // Block 0 starts accumulator 0. Later blocks switch to the other accumulator
+              // (overwriting it) when a row of the tile raised its max: the softmax warps'
+              // votes, written before their p_full arrivals.
+              bool fresh = (t == 1);
+              if (t > 1) {
+                const volatile uint32_t* vt = votes + (((t - 1) & 1) * NQ + q) * 4;
+                if ((vt[0] | vt[1] | vt[2] | vt[3]) != 0u) {
+                  cur_acc ^= 1u << q;
+                  fresh = true;
+                }
+              }
+              const uint32_t acc = tmem + C::tO(q, (cur_acc >> q) & 1u);
               const uint32_t vbase = smem_u32(sV + ((t - 1) % S) * C::kVBytes);
 #pragma unroll
               for (int kk = 0; kk < BN / 32; ++kk)
-                mma_i8_ts(tmem + C::tO(q), tmem + C::tP(q) + 8 * kk, smem_desc(vbase + 512 * kk, 128, 2048),
-                          idesc_pv, (t > 1 || kk > 0) ? 1u : 0u);
+                mma_i8_ts(acc, tmem + C::tP(q) + 8 * kk, smem_desc(vbase + 512 * kk, 128, 2048), idesc_pv,
+                          (fresh && kk == 0) ? 0u : 1u);
             }
             if (t < T) {
               if (q == 0) {
@@ -408,8 +522,9 @@ __global__ void __launch_bounds__(Cfg<DP, NQ_>::kThreads, Cfg<DP, NQ_>::kCtasPer
     const uint32_t lane_base = static_cast<uint32_t>(w4 * 32) << 16;
     const uint32_t aS = tmem + lane_base + C::tS(q);
     const uint32_t aP = tmem + lane_base + C::tP(q);
-    const uint32_t aO = tmem + lane_base + C::tO(q);
-    const uint32_t aF = tmem + lane_base + C::tF(q);
+    const uint32_t aO0 = tmem + lane_base + C::tO(q, 0);
+    const uint32_t aO1 = tmem + lane_base + C::tO(q, 1);
+    const uint32_t aF = tmem + lane_base + C::tF(q);  // unused when F is in shared memory
     const float alpha = __fmul_rn(__fmul_rn(p.softmax_scale, p.mu_q[bh]), p.mu_k[bh]);
     const float2 alpha2 = make_float2(alpha, alpha);
 
@@ -441,6 +556,10 @@ __global__ void __launch_bounds__(Cfg<DP, NQ_>::kThreads, Cfg<DP, NQ_>::kCtasPer
 
     float m = -CUDART_INF_F, l = 0.0f;
     bool alive = true;
+    // Accumulator that P.V of the current block adds into (tile-uniform), whether F holds
+    // anything yet, and how many blocks that accumulator holds.
+    int cur = 0, nblk = 1;
+    bool f_valid = false;
 
     for (int t = 0; t < T && alive; ++t) {
       const int st = t % S;
@@ -549,40 +668,36 @@ __global__ void __launch_bounds__(Cfg<DP, NQ_>::kThreads, Cfg<DP, NQ_>::kCtasPer
         }
       }
       const float lt = (lt2[0].x + lt2[0].y) + (lt2[1].x + lt2[1].y);
-      const float ct = (m == -CUDART_INF_F) ? 0.0f : ex2_approx((m - m_new) * kLog2e);
+      // Rescale factor of the row's earlier blocks: exactly 1 while its max is unchanged.
+      const float ct = (m == -CUDART_INF_F) ? 0.0f : (m_new > m ? ex2_approx((m - m_new) * kLog2e) : 1.0f);
       l = l * ct + lt;
-      // Fold the int32 accumulator into the fp32 running output F when the row max rose
-      // (t = 0: F starts at zero and P.V overwrites the accumulator).
-      const bool flush = (t > 0) && (m_new > m);
-      if (t == 0 || __any_sync(0xffffffffu, flush)) {
-#pragma unroll 1
-        for (int cc = 0; cc < DP / 16; ++cc) {
-          uint32_t a[16], f[16];
-          if (t > 0) {
-            tmem_ld16(aO + 16 * cc, a);
-            tmem_ld16(aF + 16 * cc, f);
-            tmem_ld_wait();
-            reg_fence16(a);
-            reg_fence16(f);
-          }
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            if (t == 0) {
-              f[e] = 0u;
-            } else if (flush) {
-              f[e] = __float_as_uint((__uint_as_float(f[e]) + __int2float_rn(static_cast<int>(a[e]))) * ct);
-              a[e] = 0u;
-            }
-          }
-          if (t > 0) tmem_st16(aO + 16 * cc, a);
-          tmem_st16(aF + 16 * cc, f);
-        }
-      }
+      // Vote (per warp) whether a row raised its max; the MMA thread reads the votes of the
+      // tile's four warps after their p_full arrivals.
+      const bool rose = __any_sync(0xffffffffu, t > 0 && m_new > m);
+      if (lane == 0) votes[((t & 1) * NQ + q) * 4 + w4] = rose ? 1u : 0u;
       m = m_new;
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars[Bar::pfull(q)]);
+      if (t == 0) continue;
+      // While the MMAs of the next block run: if any row of the tile raised its max, P.V of
+      // this block goes to the other accumulator, and the old one is folded into F with this
+      // row's factor (1 for rows whose max did not rise).
+      if (!wait_warp(&bars[Bar::pfull(q)], t & 1, abort_flag)) {
+        alive = false;
+        break;
+      }
+      const volatile uint32_t* vt = votes + ((t & 1) * NQ + q) * 4;
+      if ((vt[0] | vt[1] | vt[2] | vt[3]) != 0u) {
+        fold_rest<C, 0>(cur ? aO1 : aO0, aF, sF + q * BM + r, make_float2(ct, ct), !f_valid, nblk == 1);
+        if (!C::kFSmem) tmem_st_wait();
+        cur ^= 1;
+        f_valid = true;
+        nblk = 1;
+      } else {
+        ++nblk;
+      }
     }
 
     if (alive && wait_warp(&bars[Bar::odone(q)], 0, abort_flag)) {
@@ -593,18 +708,34 @@ __global__ void __launch_bounds__(Cfg<DP, NQ_>::kThreads, Cfg<DP, NQ_>::kCtasPer
       const int esz = (p.o_dt == BA_F32) ? 4 : 2;
       const bool vec = ((d * esz) & 15) == 0;
       char* orow = reinterpret_cast<char*>(p.o) + ((bh * N + i) * d) * esz;
-#pragma unroll
+      const uint32_t aO = cur ? aO1 : aO0;
+      const float4* fr = sF + q * BM + r;
+#pragma unroll 1
       for (int cc = 0; cc < DP / 16; ++cc) {
-        uint32_t a[16], f[16];
+        uint32_t a[16];
+        float f[16];
         tmem_ld16(aO + 16 * cc, a);
-        tmem_ld16(aF + 16 * cc, f);
-        tmem_ld_wait();
-        reg_fence16(a);
-        reg_fence16(f);
+        if constexpr (C::kFSmem) {
+          tmem_ld_wait();
+          reg_fence16(a);
+#pragma unroll
+          for (int k4 = 0; k4 < 4; ++k4) {
+            const float4 v = f_valid ? fr[(4 * cc + k4) * (NQ * BM)] : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+            f[4 * k4] = v.x; f[4 * k4 + 1] = v.y; f[4 * k4 + 2] = v.z; f[4 * k4 + 3] = v.w;
+          }
+        } else {
+          uint32_t fb[16];
+          if (f_valid) tmem_ld16(aF + 16 * cc, fb);
+          tmem_ld_wait();
+          reg_fence16(a);
+          if (f_valid) reg_fence16(fb);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) f[e] = f_valid ? __uint_as_float(fb[e]) : 0.0f;
+        }
         float val[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e)
-          val[e] = (__uint_as_float(f[e]) + __int2float_rn(static_cast<int>(a[e]))) * sscale[16 * cc + e] * inv_l;
+          val[e] = (f[e] + __int2float_rn(static_cast<int>(a[e]))) * sscale[16 * cc + e] * inv_l;
         if (!row_ok) continue;
         if (vec && 16 * cc + 16 <= d) {
           if (p.o_dt == BA_F32) {
@@ -701,6 +832,9 @@ cudaError_t launch_cfg(const AttnParams& p, const CUtensorMap& tm, cudaStream_t 
   static int configured = 0;
   if (smem > configured) {
     cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<DP, BK, NQ>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(attn_tc_kernel<DP, BK, NQ>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
     configured = smem;
   }
