@@ -340,34 +340,54 @@ ba_status ba_attention_fwd(const void* q, const void* k, const void* v, ba_dtype
   const PrepDims g = dims(B, H, N, d);
   std::vector<cudaEvent_t> ev = timing_events();
   record(ev, 0, s);
-  // One launch streams q, k and v: sign bits + |x| partial sums for q and k, channel
-  // maxima for v.
-  PrepParams pp{};
-  pp.g = g;
-  pp.job[0] = PrepJob{q, kJobPack, at<uint32_t>(ws, L.bits_q), at<double>(ws, L.part_mu_q), nullptr};
-  pp.job[1] = PrepJob{k, kJobPack, at<uint32_t>(ws, L.bits_k), at<double>(ws, L.part_mu_k), nullptr};
-  pp.job[2] = PrepJob{v, kJobAmax, nullptr, nullptr, at<float>(ws, L.part_amax)};
-  if ((st = cuda_status(launch_prep(pp, dt, 3, s))) != BA_OK) return keep(ev, false), st;
-  record(ev, 1, s);
-  FinalizeParams fp{};
-  fp.g = g;
-  fp.npack = 2;
-  fp.part_mu[0] = at<double>(ws, L.part_mu_q);
-  fp.part_mu[1] = at<double>(ws, L.part_mu_k);
-  fp.mu[0] = at<float>(ws, L.mu_q);
-  fp.mu[1] = at<float>(ws, L.mu_k);
-  fp.part_amax = at<float>(ws, L.part_amax);
-  fp.inv = at<float>(ws, L.inv);
-  fp.v_scale = at<float>(ws, L.v_scale);
-  if ((st = cuda_status(launch_finalize(fp, s))) != BA_OK) return keep(ev, false), st;
-  record(ev, 2, s);
-  QuantParams qp{};
-  qp.g = g;
-  qp.v = v;
-  qp.inv = at<float>(ws, L.inv);
-  qp.vq = at<int8_t>(ws, L.vq);
-  if ((st = cuda_status(launch_quant(qp, dt, s))) != BA_OK) return keep(ev, false), st;
-  record(ev, 3, s);
+  if (use_slice_prep(g)) {
+    // Many slices of whole 16-byte rows: one launch prepares q, k and v slice by slice (the
+    // finalize and quantise stages are empty).
+    SliceParams sp{};
+    sp.g = g;
+    sp.q = q;
+    sp.k = k;
+    sp.v = v;
+    sp.bits_q = at<uint32_t>(ws, L.bits_q);
+    sp.bits_k = at<uint32_t>(ws, L.bits_k);
+    sp.mu_q = at<float>(ws, L.mu_q);
+    sp.mu_k = at<float>(ws, L.mu_k);
+    sp.vq = at<int8_t>(ws, L.vq);
+    sp.v_scale = at<float>(ws, L.v_scale);
+    if ((st = cuda_status(launch_prep_slices(sp, dt, s))) != BA_OK) return keep(ev, false), st;
+    record(ev, 1, s);
+    record(ev, 2, s);
+    record(ev, 3, s);
+  } else {
+    // One launch streams q, k and v: sign bits + |x| partial sums for q and k, channel
+    // maxima for v.
+    PrepParams pp{};
+    pp.g = g;
+    pp.job[0] = PrepJob{q, kJobPack, at<uint32_t>(ws, L.bits_q), at<double>(ws, L.part_mu_q), nullptr};
+    pp.job[1] = PrepJob{k, kJobPack, at<uint32_t>(ws, L.bits_k), at<double>(ws, L.part_mu_k), nullptr};
+    pp.job[2] = PrepJob{v, kJobAmax, nullptr, nullptr, at<float>(ws, L.part_amax)};
+    if ((st = cuda_status(launch_prep(pp, dt, 3, s))) != BA_OK) return keep(ev, false), st;
+    record(ev, 1, s);
+    FinalizeParams fp{};
+    fp.g = g;
+    fp.npack = 2;
+    fp.part_mu[0] = at<double>(ws, L.part_mu_q);
+    fp.part_mu[1] = at<double>(ws, L.part_mu_k);
+    fp.mu[0] = at<float>(ws, L.mu_q);
+    fp.mu[1] = at<float>(ws, L.mu_k);
+    fp.part_amax = at<float>(ws, L.part_amax);
+    fp.inv = at<float>(ws, L.inv);
+    fp.v_scale = at<float>(ws, L.v_scale);
+    if ((st = cuda_status(launch_finalize(fp, s))) != BA_OK) return keep(ev, false), st;
+    record(ev, 2, s);
+    QuantParams qp{};
+    qp.g = g;
+    qp.v = v;
+    qp.inv = at<float>(ws, L.inv);
+    qp.vq = at<int8_t>(ws, L.vq);
+    if ((st = cuda_status(launch_quant(qp, dt, s))) != BA_OK) return keep(ev, false), st;
+    record(ev, 3, s);
+  }
 
   AttnParams ap{};
   ap.bias = bp;

@@ -46,7 +46,24 @@ struct QuantParams {
   int8_t* vq;
 };
 
+// Whole-slice preparation (one warp per (b, h) and tensor; d % 8 == 0): sign bits and mu of q
+// and k, channel scales and int8 rows of v, in one launch.
+struct SliceParams {
+  PrepDims g;
+  const void* q;
+  const void* k;
+  const void* v;
+  uint32_t* bits_q;
+  uint32_t* bits_k;
+  float* mu_q;
+  float* mu_k;
+  int8_t* vq;
+  float* v_scale;
+};
+
 cudaError_t launch_prep(const PrepParams& p, int dt, int njobs, cudaStream_t s);
+cudaError_t launch_prep_slices(const SliceParams& p, int dt, cudaStream_t s);
+bool use_slice_prep(const PrepDims& g);
 cudaError_t launch_finalize(const FinalizeParams& p, cudaStream_t s);
 cudaError_t launch_quant(const QuantParams& p, int dt, cudaStream_t s);
 

@@ -1,15 +1,20 @@
 // Streaming kernels of the BinaryAttention forward pass (sm_100a):
-//   prep_kernel     — sign bits + per-chunk sum |x| of q and k, per-chunk channel max |v|;
-//   finalize_kernel — mu = sum / (N d) per (b, h); per-channel V scales;
-//   quant_kernel    — V -> int8 rows with the per-channel inverse scale.
+//   prep_slice_kernel — short slices (d % 8 == 0, d >= 32, many slices): one CTA per (slice,
+//                       tensor) writes the sign bits and mu of q and k, or the scales and int8
+//                       rows of v, in one launch;
+//   prep_warp_kernel  — otherwise, rows of whole 16-byte pieces: one warp per 128-token chunk,
+//                       sign bits + per-chunk sum |x| of q and k, per-chunk channel max |v|;
+//   prep_kernel       — the same per chunk for any d (CTA per chunk; scalar path when d % 8 != 0);
+//   finalize_kernel   — mu = sum / (N d) per (b, h); per-channel V scales;
+//   quant_kernel      — V -> int8 rows with the per-channel inverse scale.
 // Sign binarisation and mu: gist.science/zh technical summary 2.2(1) (s_i = mu_q sign(q_i),
 // mu the mean along token and channel axes). Channel-aware 8-bit V: gist.science/zh 2.2(3),
 // gist.science/nl Methodologie 2.
 //
-// All three are HBM-bound: each 128-token chunk of one (b, h) slice is one CTA, read with
-// 16-byte non-allocating loads, fully coalesced (consecutive threads read consecutive
-// 16-byte pieces of consecutive rows). Reductions are deterministic: fixed-order in-CTA
-// trees, then fixed-order sums over chunks.
+// All are HBM-bound: 16-byte loads, fully coalesced (consecutive threads read consecutive
+// 16-byte pieces of consecutive rows), many in flight per thread. The |x| sums are taken in
+// double, where every partial sum of 16-bit magnitudes is exact, so they do not depend on the
+// summation order.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -252,9 +257,306 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(QuantParams p) {
   }
 }
 
+// ---------------------------------------------------------------------------------------
+// Warp-granular streaming for rows of whole 16-byte pieces (d % 8 == 0). A warp covers
+// rpp = 32 / (d/8) rows per pass, lane (row-in-pass, piece) reading one 16-byte piece, so a
+// pass reads rpp consecutive rows as one coalesced span; kBatch passes are loaded before any
+// is used. Warps never wait for each other: reductions are warp shuffles, and the sign bytes
+// of a chunk are assembled in the warp's own shared-memory rows.
+constexpr int kWarps = kThreads / 32;
+constexpr int kBatch = 8;
+
+struct Lanes {
+  int tpr, rpp, sub, rp;
+  bool on;
+};
+
+__device__ __forceinline__ Lanes lanes_for(int d) {
+  Lanes L;
+  const int lane = threadIdx.x & 31;
+  L.tpr = d >> 3;
+  L.rpp = 32 / L.tpr;
+  L.sub = lane % L.tpr;
+  L.rp = lane / L.tpr;
+  L.on = L.rp < L.rpp;
+  return L;
+}
+
+__device__ __forceinline__ double warp_sum(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Max over the lanes that hold the same 8 channels (lanes sub + tpr * t); every lane of the
+// group gets the result.
+__device__ __forceinline__ void group_max(float (&mx)[8], const Lanes& L) {
+  float m[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) m[e] = __shfl_sync(0xffffffffu, mx[e], L.sub);
+  for (int t = 1; t < L.rpp; ++t) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) m[e] = fmaxf(m[e], __shfl_sync(0xffffffffu, mx[e], L.sub + L.tpr * t));
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) mx[e] = m[e];
+}
+
+// Sign bytes and sum |x| of one chunk (rows [0, ntok) at `rows`, row stride d). The chunk's
+// 16-byte sign rows go to `bits` through the warp's staging rows `sb` (bytes past d/8 are
+// zero). Returns this lane's part of the sum.
+template <typename T>
+__device__ __forceinline__ double pack_chunk(const char* rows, int ntok, int d, const Lanes& L, uint8_t (*sb)[16],
+                                             uint4* bits) {
+  double acc = 0.0;
+  const int npass = (ntok + L.rpp - 1) / L.rpp;
+  for (int p0 = 0; p0 < npass; p0 += kBatch) {
+    uint4 u[kBatch];
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) {
+      const int r = (p0 + j) * L.rpp + L.rp;
+      if (L.on && r < ntok) u[j] = ldg_stream(rows + (static_cast<int64_t>(r) * d + L.sub * 8) * 2);
+    }
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) {
+      const int r = (p0 + j) * L.rpp + L.rp;
+      if (L.on && r < ntok) {
+        float f[8];
+        unpack8<T>(u[j], f);
+        uint32_t byte = 0;
+        double a8[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          byte |= (f[e] < 0.0f ? 1u : 0u) << e;
+          a8[e] = static_cast<double>(fabsf(f[e]));
+        }
+        // Every partial sum of 16-bit magnitudes is exact in double: the order is free.
+        acc += ((a8[0] + a8[1]) + (a8[2] + a8[3])) + ((a8[4] + a8[5]) + (a8[6] + a8[7]));
+        sb[r][L.sub] = static_cast<uint8_t>(byte);
+      }
+    }
+  }
+  __syncwarp();
+  for (int r = threadIdx.x & 31; r < ntok; r += 32) bits[r] = *reinterpret_cast<const uint4*>(sb[r]);
+  __syncwarp();
+  return acc;
+}
+
+// Channel maxima |v| of one chunk into this lane's 8 channels (8 * sub ...).
+template <typename T>
+__device__ __forceinline__ void amax_chunk(const char* rows, int ntok, int d, const Lanes& L, float (&mx)[8]) {
+  const int npass = (ntok + L.rpp - 1) / L.rpp;
+  for (int p0 = 0; p0 < npass; p0 += kBatch) {
+    uint4 u[kBatch];
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) {
+      const int r = (p0 + j) * L.rpp + L.rp;
+      if (L.on && r < ntok) u[j] = __ldg(reinterpret_cast<const uint4*>(rows + (static_cast<int64_t>(r) * d + L.sub * 8) * 2));
+    }
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) {
+      const int r = (p0 + j) * L.rpp + L.rp;
+      if (L.on && r < ntok) {
+        float f[8];
+        unpack8<T>(u[j], f);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) mx[e] = fmaxf(mx[e], fabsf(f[e]));
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ uint8_t (*warp_bits_rows())[16] {
+  __shared__ __align__(16) uint8_t sbits[kWarps][kPrepTokens][16];
+  uint8_t (*sb)[16] = sbits[threadIdx.x >> 5];
+  // Bytes past d/8 of a sign row are never written: zero this warp's rows once.
+  for (int e = threadIdx.x & 31; e < kPrepTokens; e += 32) *reinterpret_cast<uint4*>(sb[e]) = make_uint4(0u, 0u, 0u, 0u);
+  __syncwarp();
+  return sb;
+}
+
+// Chunk mode: one warp per (job, slice, 128-token chunk); per-chunk partials for finalize.
+template <typename T>
+__global__ void __launch_bounds__(kThreads, 3) prep_warp_kernel(PrepParams p, int njobs) {
+  const PrepDims& g = p.g;
+  const int64_t per_job = g.BH * g.nchunk;
+  const int64_t unit = static_cast<int64_t>(blockIdx.x) * kWarps + (threadIdx.x >> 5);
+  uint8_t (*sb)[16] = warp_bits_rows();
+  if (unit >= njobs * per_job) return;
+  const int j = static_cast<int>(unit / per_job);
+  const PrepJob job = j == 0 ? p.job[0] : (j == 1 ? p.job[1] : p.job[2]);
+  const int64_t rest = unit - j * per_job;
+  const int64_t bh = rest / g.nchunk;
+  const int chunk = static_cast<int>(rest - bh * g.nchunk);
+  const int tok0 = chunk * kPrepTokens;
+  const int ntok = min(kPrepTokens, g.N - tok0);
+  const Lanes L = lanes_for(g.d);
+  const char* rows = reinterpret_cast<const char*>(job.src) + ((bh * g.N + tok0) * g.d) * 2;
+  if (job.kind == kJobPack) {
+    const double tot = warp_sum(pack_chunk<T>(rows, ntok, g.d, L, sb, reinterpret_cast<uint4*>(job.bits) + bh * g.N + tok0));
+    if ((threadIdx.x & 31) == 0) job.part_sum[bh * g.nchunk + chunk] = tot;
+  } else {
+    float mx[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) mx[e] = 0.0f;
+    amax_chunk<T>(rows, ntok, g.d, L, mx);
+    group_max(mx, L);
+    if (L.on && L.rp == 0) {
+      float* out = job.part + (bh * g.nchunk + chunk) * g.dp + L.sub * 8;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) out[e] = mx[e];
+      if ((g.d & 15) == 8 && L.sub == L.tpr - 1)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) out[8 + e] = 0.0f;
+    }
+  }
+}
+
+// Whole-slice mode (d >= 32): one CTA per (slice, tensor) loads the slice in batches of kSliceBatch
+// passes of rpp = 256 / (d/8) rows (a slice of up to kSliceBatch * rpp rows in one batch, all of
+// its loads in flight at once), then reduces once: mu for q and k; for v the channel maxima, the
+// scales, and a second batch of loads (L2) that quantises. Sign bytes are assembled per batch
+// in shared memory and written as 16-byte rows.
+constexpr int kSliceBatch = 10;
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads, 3) prep_slice_kernel(SliceParams p) {
+  __shared__ __align__(16) uint8_t sbits[kSliceBatch * kThreads / 4][16];  // d >= 32: at most 64 rows per pass
+  __shared__ float smax[kThreads * 8];
+  __shared__ double sred[kThreads / 32];
+  const PrepDims& g = p.g;
+  const int64_t bh = blockIdx.x;
+  const int job = blockIdx.y;  // 0: q, 1: k, 2: v
+  const int d = g.d, dp = g.dp;
+  const int tpr = d >> 3;
+  const int rpp = kThreads / tpr;
+  const int sub = threadIdx.x % tpr, rp = threadIdx.x / tpr;
+  const bool on = rp < rpp;
+  const int rows_per_batch = kSliceBatch * rpp;
+  const char* src = reinterpret_cast<const char*>(job == 0 ? p.q : (job == 1 ? p.k : p.v)) + (bh * g.N * d) * 2;
+  if (job < 2) {
+    // Bytes past d/8 of a sign row are never written.
+    for (int e = threadIdx.x; e < rows_per_batch; e += kThreads)
+      *reinterpret_cast<uint4*>(sbits[e]) = make_uint4(0u, 0u, 0u, 0u);
+    __syncthreads();
+    uint4* bits = reinterpret_cast<uint4*>(job == 0 ? p.bits_q : p.bits_k) + bh * g.N;
+    double acc = 0.0;
+    for (int r0 = 0; r0 < g.N; r0 += rows_per_batch) {
+      const int nrow = min(rows_per_batch, g.N - r0);
+      uint4 u[kSliceBatch];
+#pragma unroll
+      for (int j = 0; j < kSliceBatch; ++j) {
+        const int r = j * rpp + rp;
+        if (on && r < nrow) u[j] = ldg_stream(src + (static_cast<int64_t>(r0 + r) * d + sub * 8) * 2);
+      }
+#pragma unroll
+      for (int j = 0; j < kSliceBatch; ++j) {
+        const int r = j * rpp + rp;
+        if (on && r < nrow) {
+          float f[8];
+          unpack8<T>(u[j], f);
+          uint32_t byte = 0;
+          double a8[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            byte |= (f[e] < 0.0f ? 1u : 0u) << e;
+            a8[e] = static_cast<double>(fabsf(f[e]));
+          }
+          // Every partial sum of 16-bit magnitudes is exact in double: the order is free.
+          acc += ((a8[0] + a8[1]) + (a8[2] + a8[3])) + ((a8[4] + a8[5]) + (a8[6] + a8[7]));
+          sbits[r][sub] = static_cast<uint8_t>(byte);
+        }
+      }
+      __syncthreads();
+      for (int r = threadIdx.x; r < nrow; r += kThreads) bits[r0 + r] = *reinterpret_cast<const uint4*>(sbits[r]);
+      __syncthreads();
+    }
+    const double tot = block_sum(acc, sred);
+    if (threadIdx.x == 0) (job == 0 ? p.mu_q : p.mu_k)[bh] = static_cast<float>(tot / (static_cast<double>(g.N) * d));
+    return;
+  }
+  // v: channel maxima over the slice.
+  float mx[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) mx[e] = 0.0f;
+  for (int r0 = 0; r0 < g.N; r0 += rows_per_batch) {
+    const int nrow = min(rows_per_batch, g.N - r0);
+    uint4 u[kSliceBatch];
+#pragma unroll
+    for (int j = 0; j < kSliceBatch; ++j) {
+      const int r = j * rpp + rp;
+      if (on && r < nrow) u[j] = __ldg(reinterpret_cast<const uint4*>(src + (static_cast<int64_t>(r0 + r) * d + sub * 8) * 2));
+    }
+#pragma unroll
+    for (int j = 0; j < kSliceBatch; ++j) {
+      const int r = j * rpp + rp;
+      if (on && r < nrow) {
+        float f[8];
+        unpack8<T>(u[j], f);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) mx[e] = fmaxf(mx[e], fabsf(f[e]));
+      }
+    }
+  }
+  __shared__ float sinv[128];
+  if (on) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) smax[rp * d + sub * 8 + e] = mx[e];
+  }
+  __syncthreads();
+  const int rows = min(rpp, g.N);
+  for (int c = threadIdx.x; c < dp; c += kThreads) {
+    float m = 0.0f;
+    if (c < d)
+      for (int rr = 0; rr < rows; ++rr) m = fmaxf(m, smax[rr * d + c]);
+    const bool live = (c < d) && (m > 0.0f);
+    sinv[c] = live ? __fdiv_rn(127.0f, m) : 0.0f;
+    if (c < d) p.v_scale[bh * d + c] = live ? __fdiv_rn(m, 127.0f) : 0.0f;
+  }
+  __syncthreads();
+  float inv[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) inv[e] = sinv[sub * 8 + e];
+  const bool pad = (d & 15) == 8 && sub == tpr - 1;
+  int8_t* vq = p.vq + bh * g.N * dp;
+  for (int r0 = 0; r0 < g.N; r0 += rows_per_batch) {
+    const int nrow = min(rows_per_batch, g.N - r0);
+    uint4 u[kSliceBatch];
+#pragma unroll
+    for (int j = 0; j < kSliceBatch; ++j) {
+      const int r = j * rpp + rp;
+      if (on && r < nrow) u[j] = ldg_stream(src + (static_cast<int64_t>(r0 + r) * d + sub * 8) * 2);
+    }
+#pragma unroll
+    for (int j = 0; j < kSliceBatch; ++j) {
+      const int r = j * rpp + rp;
+      if (on && r < nrow) {
+        float f[8];
+        unpack8<T>(u[j], f);
+        const uint2 w = make_uint2(quant4(f, inv), quant4(f + 4, inv + 4));
+        int8_t* o = vq + static_cast<int64_t>(r0 + r) * dp + sub * 8;
+        if (pad)
+          *reinterpret_cast<uint4*>(o) = make_uint4(w.x, w.y, 0u, 0u);
+        else
+          *reinterpret_cast<uint2*>(o) = w;
+      }
+    }
+  }
+}
+
 }  // namespace
 
+unsigned warp_grid(int64_t units) { return static_cast<unsigned>(ceil_div(units, kWarps)); }
+
 cudaError_t launch_prep(const PrepParams& p, int dt, int njobs, cudaStream_t s) {
+  if ((p.g.d & 7) == 0) {
+    const unsigned grid = warp_grid(njobs * p.g.BH * p.g.nchunk);
+    if (dt == BA_F16)
+      prep_warp_kernel<__half><<<grid, kThreads, 0, s>>>(p, njobs);
+    else
+      prep_warp_kernel<__nv_bfloat16><<<grid, kThreads, 0, s>>>(p, njobs);
+    return cudaGetLastError();
+  }
   const dim3 grid(static_cast<unsigned>(p.g.BH * p.g.nchunk), static_cast<unsigned>(njobs));
   if (dt == BA_F16)
     prep_kernel<__half><<<grid, kThreads, 0, s>>>(p);
@@ -265,6 +567,25 @@ cudaError_t launch_prep(const PrepParams& p, int dt, int njobs, cudaStream_t s) 
 
 cudaError_t launch_finalize(const FinalizeParams& p, cudaStream_t s) {
   finalize_kernel<<<static_cast<unsigned>(p.g.BH), 128, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+// The whole-slice kernel gives each CTA a whole (slice, tensor): it needs enough slices to fill
+// the GPU and short slices (at most two load batches each; longer ones stream better as
+// 128-token chunks spread over many CTAs), and rows of whole 16-byte pieces.
+bool use_slice_prep(const PrepDims& g) {
+  if ((g.d & 7) != 0 || g.d < 32) return false;
+  const int rows_per_batch = kSliceBatch * (kThreads / (g.d >> 3));
+  return 3 * g.BH >= 384 && g.N <= 2 * rows_per_batch;
+}
+
+cudaError_t launch_prep_slices(const SliceParams& p, int dt, cudaStream_t s) {
+  if ((p.g.d & 7) != 0 || p.g.d < 32) return cudaErrorInvalidValue;
+  const dim3 grid(static_cast<unsigned>(p.g.BH), 3);
+  if (dt == BA_F16)
+    prep_slice_kernel<__half><<<grid, kThreads, 0, s>>>(p);
+  else
+    prep_slice_kernel<__nv_bfloat16><<<grid, kThreads, 0, s>>>(p);
   return cudaGetLastError();
 }
 
