@@ -346,6 +346,27 @@ __global__ void __launch_bounds__(Cfg<DP, NQ_>::kThreads, Cfg<DP, NQ_>::kCtasPer
     fence_proxy_async_smem();
     tma_prefetch_desc(&tmap_v);
   }
+  // Warps 2 and 3 load the sign rows of their Q rows and of key block 0 before the setup barrier,
+  // so the loads overlap the setup.
+  const uint4 zero4 = make_uint4(0u, 0u, 0u, 0u);
+  uint4 pre_q[NQ][2], pre_k[2];
+  if (warp == 2 || warp == 3) {
+    const int half = warp - 2;
+    const uint4* qrows = reinterpret_cast<const uint4*>(p.bits_q) + bh * N;
+    const uint4* krows = reinterpret_cast<const uint4*>(p.bits_k) + bh * N;
+#pragma unroll
+    for (int q = 0; q < NQ; ++q)
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int row = q0 + q * BM + 64 * half + lane + 32 * u;
+        pre_q[q][u] = row < N ? __ldg(qrows + row) : zero4;
+      }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int row = 64 * half + lane + 32 * u;
+      pre_k[u] = row < N ? __ldg(krows + row) : zero4;
+    }
+  }
   if (threadIdx.x < 128)
     sscale[threadIdx.x] = (threadIdx.x < d) ? p.v_scale[bh * d + threadIdx.x] * (1.0f / 255.0f) : 0.0f;
   if (is_relpos(BK) && tab_mode != 0) {
@@ -403,30 +424,17 @@ __global__ void __launch_bounds__(Cfg<DP, NQ_>::kThreads, Cfg<DP, NQ_>::kCtasPer
     // Warp 2 expands rows 0..63 and warp 3 rows 64..127 of every Q tile and K block. The
     // sign rows of the next block are loaded into registers before this block is written.
     const int half = warp - 2;
-    const uint4* qrows = reinterpret_cast<const uint4*>(p.bits_q) + bh * N;
     const uint4* krows = reinterpret_cast<const uint4*>(p.bits_k) + bh * N;
-    const uint4 zero4 = make_uint4(0u, 0u, 0u, 0u);
-    for (int q = 0; q < NQ; ++q) {
-      uint4 b[2];
-      bool ok[2];
 #pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int row = q0 + q * BM + 64 * half + lane + 32 * u;
-        ok[u] = row < N;
-        b[u] = ok[u] ? __ldg(qrows + row) : zero4;
-      }
+    for (int q = 0; q < NQ; ++q)
 #pragma unroll
-      for (int u = 0; u < 2; ++u) expand_row<DQ>(sQ + q * C::kQBytes, b[u], ok[u], 64 * half + lane + 32 * u, d);
-    }
+      for (int u = 0; u < 2; ++u)
+        expand_row<DQ>(sQ + q * C::kQBytes, pre_q[q][u], q0 + q * BM + 64 * half + lane + 32 * u < N,
+                       64 * half + lane + 32 * u, d);
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) mbar_arrive(&bars[Bar::qfull()]);
-    uint4 nb[2];
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int row = 64 * half + lane + 32 * u;
-      nb[u] = row < N ? __ldg(krows + row) : zero4;
-    }
+    uint4 nb[2] = {pre_k[0], pre_k[1]};
     for (int t = 0; t < T; ++t) {
       const int st = t % S;
       const uint4 cb[2] = {nb[0], nb[1]};
