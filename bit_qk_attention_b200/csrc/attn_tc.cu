@@ -209,6 +209,38 @@ __device__ __forceinline__ void fast_block(uint32_t (&x)[32], int c, int nk, flo
   }
 }
 
+// 2^t for a pair of t <= 0 on the FMA and integer pipes, for the share of the softmax's
+// exponentials that the transcendental unit (which computes the rest, and is the softmax's
+// bottleneck) does not take. t is clamped to -125 (2^-125: a u8 code of 0, a negligible
+// addition to the row sum; masked keys arrive as -inf); j = rint(t) by adding and subtracting
+// 1.5 * 2^23, f = t - j in [-1/2, 1/2]; 2^f by a degree-5 polynomial with c0 = 1 (a weighted
+// least-squares fit in relative error on Chebyshev nodes, bit_qk_attention_b200/exp2_poly.py;
+// at most 1.6e-7 relative error in float32); 2^j is added to the exponent bits: the bit
+// pattern of t + 1.5 * 2^23 holds j in its low bits, and shifted left by 23 it is j << 23.
+__device__ __forceinline__ float2 exp2_poly2(float2 t) {
+  t.x = fmaxf(t.x, -125.0f);
+  t.y = fmaxf(t.y, -125.0f);
+  const float2 r = __fadd2_rn(t, make_float2(12582912.0f, 12582912.0f));
+  const float2 j = __fadd2_rn(r, make_float2(-12582912.0f, -12582912.0f));
+  const float2 f = __ffma2_rn(j, make_float2(-1.0f, -1.0f), t);
+  float2 q = __ffma2_rn(make_float2(1.321867225e-03f, 1.321867225e-03f), f,
+                        make_float2(9.671698324e-03f, 9.671698324e-03f));
+  q = __ffma2_rn(q, f, make_float2(5.550893024e-02f, 5.550893024e-02f));
+  q = __ffma2_rn(q, f, make_float2(2.402223796e-01f, 2.402223796e-01f));
+  q = __ffma2_rn(q, f, make_float2(6.931468844e-01f, 6.931468844e-01f));
+  q = __ffma2_rn(q, f, make_float2(1.0f, 1.0f));
+  return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(r.x) << 23)),
+                     __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(r.y) << 23)));
+}
+
+// Pairs (of the 16 in a 32-key chunk) whose exponentials take the polynomial: the bits of
+// kPolyPairs, spread over the chunk. A quarter measured fastest on B200 (more moves the limit
+// to instruction issue).
+#ifndef BA_POLY_PAIRS
+#define BA_POLY_PAIRS 0x8888u
+#endif
+constexpr uint32_t kPolyPairs = BA_POLY_PAIRS;
+
 // Folding an s32 P.V accumulator row into the fp32 running output of the row:
 // F = (F + acc) * ct, in groups of NC chunks of 16 columns starting at chunk C0. fold_load
 // issues a group's tensor-memory loads (the accumulator, and F when it lives in tensor
@@ -662,7 +694,8 @@ __global__ void __launch_bounds__(Cfg<DP, NQ_>::kThreads, Cfg<DP, NQ_>::kCtasPer
               // s - m first (exact near the max), then the scale to base 2.
               const float2 t2 = __fmul2_rn(
                   __fadd2_rn(make_float2(__uint_as_float(x[u]), __uint_as_float(x[u + 1])), negm2), log2e2);
-              const float2 p2 = make_float2(ex2_approx(t2.x), ex2_approx(t2.y));
+              const float2 p2 = ((kPolyPairs >> (2 * w + e2)) & 1u) ? exp2_poly2(t2)
+                                                                    : make_float2(ex2_approx(t2.x), ex2_approx(t2.y));
               lt2[e2] = __fadd2_rn(lt2[e2], p2);
               // 255 P~ + 1.5 * 2^23: one rounding to the nearest integer (ties to even); the
               // integer sits in the low byte of the result (P~ <= 1).
