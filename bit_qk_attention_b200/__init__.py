@@ -49,6 +49,7 @@ SIGNATURES = {
     "ba_sign_words": (_I, [_I]),
     "ba_v_row_bytes": (_I, [_I]),
     "ba_kv_block": (_I, []),
+    "ba_prep_fused": (_I, [_I, _I, _I, _I]),
     "ba_pack_workspace_bytes": (_SZ, [_I, _I, _I, _I]),
     "ba_quant_workspace_bytes": (_SZ, [_I, _I, _I, _I]),
     "ba_workspace_bytes": (_SZ, [_I, _I, _I, _I]),
@@ -162,6 +163,11 @@ def v_row_bytes(d: int) -> int:
 
 def kv_block() -> int:
     return lib().ba_kv_block()
+
+
+def prep_fused(B: int, H: int, N: int, d: int) -> bool:
+    """Whether attention_fwd prepares q, k, v in one launch for this shape (see ba_prep_fused)."""
+    return bool(lib().ba_prep_fused(B, H, N, d))
 
 
 def workspace_bytes(B: int, H: int, N: int, d: int) -> int:

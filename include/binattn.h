@@ -78,6 +78,15 @@ int ba_v_row_bytes(int d);
 /* Key block of the online softmax: the 8-bit P codes depend on it (128). */
 int ba_kv_block(void);
 
+/*
+ * Preparation path ba_attention_fwd takes for this shape: 1 = one launch (one CTA per (b, h)
+ * slice and tensor writes the sign bits and mu of q and k and the scales and int8 rows of v;
+ * taken for many short slices with d a multiple of 8 and d >= 32), 0 = three launches
+ * (128-token chunks with partial sums, a finalize kernel, the V quantiser). A host query: it
+ * launches nothing and reports the choice only; both paths compute the same values.
+ */
+int ba_prep_fused(int B, int H, int N, int d);
+
 /* Workspace sizes in bytes (0 for empty problems; -1 cast to size_t for unsupported d). */
 size_t ba_pack_workspace_bytes(int B, int H, int N, int d);
 size_t ba_quant_workspace_bytes(int B, int H, int N, int d);

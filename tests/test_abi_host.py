@@ -51,6 +51,11 @@ def test_host_queries(L):
     assert L.ba_sign_words(0) == 0 and L.ba_sign_words(129) == 0
     assert [L.ba_v_row_bytes(d) for d in (1, 16, 17, 64, 72, 128)] == [16, 16, 32, 64, 80, 128]
     assert L.ba_kv_block() == 128
+    # one-launch preparation: many short slices of whole 16-byte rows
+    assert L.ba_prep_fused(64, 12, 197, 64) == 1 and L.ba_prep_fused(32, 16, 256, 72) == 1
+    assert L.ba_prep_fused(1, 16, 4096, 64) == 0 and L.ba_prep_fused(64, 12, 197, 60) == 0
+    assert L.ba_prep_fused(64, 12, 197, 16) == 0 and L.ba_prep_fused(0, 12, 197, 64) == 0
+    assert L.ba_prep_fused(64, 12, 197, 129) == 0
     assert L.ba_workspace_bytes(0, 4, 16, 64) == 0 and L.ba_workspace_bytes(2, 4, 0, 64) == 0
     big = L.ba_workspace_bytes(2, 16, 4096, 64)
     assert big >= 2 * 16 * 4096 * (16 + 16 + 64)
