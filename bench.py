@@ -382,7 +382,8 @@ def main():
             "roofline": roof,
             "cpu_baseline": cpu,
             "e2e": e2e,
-            "gpu_launches": 4 * args.steps,
+            # prep (1 launch on the one-launch path, else prep + finalize + quantise) + attention
+            "gpu_launches": ((2 if ba.prep_fused(w.B, w.H, w.N, w.d) else 4) * args.steps),
             "clocks": clk,
         }
         print(json.dumps(line), flush=True)
