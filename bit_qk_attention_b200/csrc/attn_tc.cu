@@ -7,8 +7,14 @@
 // on every page).
 //
 // How, on B200:
-//   * Each CTA owns NQ query tiles of 128 rows of one (b, h): one tile in 256 tensor-memory
+//   * A work item is NQ query tiles of 128 rows of one (b, h): one tile in 256 tensor-memory
 //     columns (two CTAs per SM) when the head and the bias table fit, else two tiles in 512.
+//     For heads up to 80 channels the CTAs are persistent (as many as fit at once): each walks
+//     a list of items, grouped by head when the head's rel-pos table is staged, while its
+//     producers and MMA thread run ahead into the next item (the K/V ring continues across
+//     items; consecutive items start on alternate P.V accumulators, so an item's epilogue
+//     overlaps the next item's first MMAs). Wider heads run one item per CTA
+//     (attn_tc_single_kernel), which measured faster there.
 //   * Warps 2 and 3 expand the 1-bit sign rows of Q (once) and of each K block into fp8 +-1
 //     operands in shared memory (channels >= d become 0); warp 0 TMA-loads the int8 V block
 //     (a 4-D tensor map that lands it in the MN-major core-matrix layout the MMA reads) and
@@ -32,6 +38,7 @@
 #include <cuda.h>
 #include <math_constants.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "common.cuh"
@@ -67,9 +74,9 @@ struct Cfg {
   static constexpr int offK = offQ + NQ * kQBytes;
   static constexpr int offV = offK + kStages * kKBytes;
   static constexpr int offKoff = offV + kStages * kVBytes;
-  static constexpr int offScale = offKoff + kStages * BN * 4;
+  static constexpr int offScale = offKoff + kStages * BN * 4;  // V scales (single-item kernel)
   static constexpr int offBar = offScale + 128 * 4;
-  static constexpr int kNumBars = 2 * kStages + 2 + 3 * NQ;
+  static constexpr int kNumBars = 2 * kStages + 3 + 3 * NQ;
   static constexpr int offMisc = offBar + kNumBars * 8;           // tmem base, abort flag
   static constexpr int offVotes = offMisc + 16;                    // [2][NQ][4] u32
   static constexpr int offF = (offVotes + 2 * NQ * 4 * 4 + 15) / 16 * 16;
@@ -94,16 +101,46 @@ struct Cfg {
   static constexpr int kCtasPerSm = 512 / kTmemCols;
 };
 
-// Barrier slots: kv_full[S], kv_empty[S], q_full, drain, s_full[NQ], p_full[NQ], o_done[NQ].
+// Barrier slots: kv_full[S], kv_empty[S], q_full, q_empty, drain, s_full[NQ], p_full[NQ],
+// o_done[NQ]. Phases count K/V blocks (kv_*: per stage; s_full, p_full: per block) or work
+// items (q_*, o_done) across all the items a CTA processes.
 template <int S, int NQ> struct Bars {
   __host__ __device__ static constexpr int kvfull(int s) { return s; }
   __host__ __device__ static constexpr int kvempty(int s) { return S + s; }
   __host__ __device__ static constexpr int qfull() { return 2 * S; }
-  __host__ __device__ static constexpr int drain() { return 2 * S + 1; }
-  __host__ __device__ static constexpr int sfull(int q) { return 2 * S + 2 + q; }
-  __host__ __device__ static constexpr int pfull(int q) { return 2 * S + 2 + NQ + q; }
-  __host__ __device__ static constexpr int odone(int q) { return 2 * S + 2 + 2 * NQ + q; }
+  __host__ __device__ static constexpr int qempty() { return 2 * S + 1; }
+  __host__ __device__ static constexpr int drain() { return 2 * S + 2; }
+  __host__ __device__ static constexpr int sfull(int q) { return 2 * S + 3 + q; }
+  __host__ __device__ static constexpr int pfull(int q) { return 2 * S + 3 + NQ + q; }
+  __host__ __device__ static constexpr int odone(int q) { return 2 * S + 3 + 2 * NQ + q; }
 };
+
+// Work items: NQ query tiles of one (b, h). With the head's rel-pos table staged in shared
+// memory (by_head), the CTAs of head h are h, h + H, h + 2H, ... (gridDim.x = H * k) and CTA j
+// of head h takes items j, j + k, j + 2k, ... of the B * nqb items of that head (nqb = query
+// blocks per (b, h)), so the table is staged once. Otherwise CTA c takes items c, c + G,
+// c + 2G, ... of all B * H * nqb items (G = gridDim.x), item m covering query block m % nqb of
+// slice m / nqb. Recomputed from the launch geometry where needed.
+__device__ __forceinline__ int item_count(bool by_head, int B, int H, int nqb) {
+  const int total = by_head ? B * nqb : B * H * nqb;
+  const int first = by_head ? static_cast<int>(blockIdx.x) / H : static_cast<int>(blockIdx.x);
+  const int stride = by_head ? static_cast<int>(gridDim.x) / H : static_cast<int>(gridDim.x);
+  return first < total ? (total - first + stride - 1) / stride : 0;
+}
+
+__device__ __forceinline__ void item_at(bool by_head, int it, int H, int nqb, int rows_per_item, int64_t& bh,
+                                        int& q0) {
+  if (by_head) {
+    const int m = static_cast<int>(blockIdx.x) / H + it * (static_cast<int>(gridDim.x) / H);
+    const int b = m / nqb;
+    bh = static_cast<int64_t>(b) * H + static_cast<int>(blockIdx.x) % H;
+    q0 = (m - b * nqb) * rows_per_item;
+  } else {
+    const int64_t m = static_cast<int64_t>(blockIdx.x) + static_cast<int64_t>(it) * gridDim.x;
+    bh = m / nqb;
+    q0 = static_cast<int>(m - bh * nqb) * rows_per_item;
+  }
+}
 
 // Waits for the phase of `bar` with the given parity. Gives up after kTimeoutNs (recording the
 // timeout in the device status word and raising the CTA's abort flag) or, when `yield` is set,
@@ -255,8 +292,9 @@ constexpr uint32_t kPolyPairs = BA_POLY_PAIRS;
 template <class C>
 struct FoldShape {
   static constexpr int NCH = C::kVBytes / BN / 16;  // chunks per row
-  // 2 chunks per group when F is in shared memory (those CTAs share an SM: 128 registers per
-  // thread), 4 when it is in tensor memory.
+  // 2 chunks (32 columns) per group when F is in shared memory (those CTAs share an SM: 128
+  // 2 chunks (32 columns) per group when F is in shared memory (those CTAs share an SM: 128
+  // registers per thread), 4 when it is in tensor memory (one CTA per SM).
   static constexpr int G = C::kFSmem ? 2 : 4;
   __host__ __device__ static constexpr int nc(int c0) { return (NCH - c0 < G) ? NCH - c0 : G; }
 };
@@ -333,6 +371,586 @@ __device__ __forceinline__ void fold_rest(uint32_t acc, uint32_t aF, float4* fr,
 template <int DP, int BK, int NQ_>
 __global__ void __launch_bounds__(Cfg<DP, NQ_>::kThreads, Cfg<DP, NQ_>::kCtasPerSm)
     attn_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmap_v, int tab_mode, int tsize,
+                   int kmax) {
+  using C = Cfg<DP, NQ_>;
+  constexpr int NQ = C::NQ, DQ = C::DQ, S = C::kStages;
+  using Bar = Bars<S, NQ>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem + C::offQ;
+  uint8_t* sK = smem + C::offK;
+  uint8_t* sV = smem + C::offV;
+  int* koff = reinterpret_cast<int*>(smem + C::offKoff);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::offBar);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::offMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::offMisc + 4);
+  // Per block parity, tile and softmax warp: whether a row of that warp raised its max.
+  uint32_t* votes = reinterpret_cast<uint32_t*>(smem + C::offVotes);
+  float4* sF = reinterpret_cast<float4*>(smem + C::offF);  // [DP/4][NQ*128]
+  // Rel-pos table of this CTA's head, staged when it fits: tab_mode 1 = table only,
+  // 2 = table followed by 2*tsize zeros (targets of prefix rows and prefix keys).
+  float* stab = reinterpret_cast<float*>(smem + C::kTabOff);
+
+  const int N = p.N, d = p.d;
+  const int nqb = static_cast<int>(ceil_div(N, BM * NQ));
+  // Items grouped by head when the head's rel-pos table is staged in shared memory.
+  const bool by_head = is_relpos(BK) && tab_mode != 0;
+  const int n_items = item_count(by_head, p.B, p.H, nqb);
+  const int T = static_cast<int>(ceil_div(N, BN));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < C::kStages; ++st) {
+      // kv_full: the V copy's expect_tx arrival + warp 0 (key offsets) + the two expanding warps.
+      mbar_init(&bars[Bar::kvfull(st)], 4);
+      mbar_init(&bars[Bar::kvempty(st)], 1);
+    }
+    mbar_init(&bars[Bar::qfull()], 2);
+    mbar_init(&bars[Bar::qempty()], 1);
+    mbar_init(&bars[Bar::drain()], 1);
+    for (int q = 0; q < NQ; ++q) {
+      mbar_init(&bars[Bar::sfull(q)], 1);
+      mbar_init(&bars[Bar::pfull(q)], 4);
+      mbar_init(&bars[Bar::odone(q)], 1);
+    }
+    *abort_flag = 0;
+    mbar_fence_init();
+    fence_proxy_async_smem();
+    tma_prefetch_desc(&tmap_v);
+  }
+  // Warps 2 and 3 load the sign rows of their Q rows and of key block 0 of the first item
+  // before the setup barrier, so the loads overlap the setup.
+  const uint4 zero4 = make_uint4(0u, 0u, 0u, 0u);
+  uint4 pre_q[NQ][2], pre_k[2];
+  if ((warp == 2 || warp == 3) && n_items > 0) {
+    const int half = warp - 2;
+    int64_t bh;
+    int q0;
+    item_at(by_head, 0, p.H, nqb, BM * NQ, bh, q0);
+    const uint4* qrows = reinterpret_cast<const uint4*>(p.bits_q) + bh * N;
+    const uint4* krows = reinterpret_cast<const uint4*>(p.bits_k) + bh * N;
+#pragma unroll
+    for (int q = 0; q < NQ; ++q)
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int row = q0 + q * BM + 64 * half + lane + 32 * u;
+        pre_q[q][u] = row < N ? __ldg(qrows + row) : zero4;
+      }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int row = 64 * half + lane + 32 * u;
+      pre_k[u] = row < N ? __ldg(krows + row) : zero4;
+    }
+  }
+  if (by_head) {
+    const float* src = p.bias.data + static_cast<int64_t>(blockIdx.x % p.H) * tsize;
+    const int n = (tab_mode == 2) ? 3 * tsize : tsize;
+    for (int e = threadIdx.x; e < n; e += C::kThreads) stab[e] = (e < tsize) ? __ldg(src + e) : 0.0f;
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer: V blocks, key offsets
+    // Blocks are counted across the items (g): stage g % S, phase g / S.
+    const int W2 = 2 * p.bias.table_w - 1;
+    int g = 0;
+    bool ok = true;
+    for (int it = 0; it < n_items && ok; ++it) {
+      int64_t bh;
+      int q0;
+      item_at(by_head, it, p.H, nqb, BM * NQ, bh, q0);
+      for (int t = 0; t < T; ++t, ++g) {
+        const int st = g % S;
+        if (g >= S && !wait_warp(&bars[Bar::kvempty(st)], ((g / S) - 1) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&bars[Bar::kvfull(st)], C::kVBytes);
+          tma_load_4d(sV + st * C::kVBytes, &tmap_v, &bars[Bar::kvfull(st)], 0, t * BN, 0, static_cast<int>(bh));
+        }
+        if (is_relpos(BK)) {
+#pragma unroll
+          for (int u = 0; u < BN / 32; ++u) {
+            const int j = lane + 32 * u, tok = t * BN + j;
+            // Keys past N read a valid entry (their P is masked); prefix keys read the zeros
+            // after the staged table (or are marked -1 for the general path).
+            int v = (tab_mode == 2) ? -tsize : -1;
+            if (tok >= N) {
+              v = 0;
+            } else if (tok >= p.bias.n_prefix) {
+              const int tj = tok - p.bias.n_prefix;
+              const int yj = tj / p.bias.grid_w;
+              v = yj * W2 + (tj - yj * p.bias.grid_w);
+            }
+            koff[st * BN + j] = 4 * v;  // byte offset into the staged table
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[Bar::kvfull(st)]);
+      }
+    }
+    // Leave no TMA copy in flight: wait (bounded, even after an abort) for the stages this
+    // warp filled last.
+    for (int k = (g > S ? g - S : 0); k < g; ++k) wait_bounded(&bars[Bar::kvfull(k % S)], (k / S) & 1, abort_flag, false);
+  } else if (warp == 2 || warp == 3) {
+    // ------------------------------------------------------------ producer: sign expansion
+    // Warp 2 expands rows 0..63 and warp 3 rows 64..127 of every Q tile and K block. The sign
+    // rows of the next K block are loaded into registers before this block is written. The Q
+    // tiles of an item are written once the MMAs of the previous item have read them (q_empty).
+    const int half = warp - 2;
+    int g = 0;
+    bool ok = true;
+    uint4 nb[2] = {pre_k[0], pre_k[1]};
+    for (int it = 0; it < n_items && ok; ++it) {
+      int64_t bh;
+      int q0;
+      item_at(by_head, it, p.H, nqb, BM * NQ, bh, q0);
+      if (it > 0) {
+        const uint4* qrows = reinterpret_cast<const uint4*>(p.bits_q) + bh * N;
+#pragma unroll
+        for (int q = 0; q < NQ; ++q)
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int row = q0 + q * BM + 64 * half + lane + 32 * u;
+            pre_q[q][u] = row < N ? __ldg(qrows + row) : zero4;
+          }
+        if (!wait_warp(&bars[Bar::qempty()], (it - 1) & 1, abort_flag)) break;
+      }
+#pragma unroll
+      for (int q = 0; q < NQ; ++q)
+#pragma unroll
+        for (int u = 0; u < 2; ++u)
+          expand_row<DQ>(sQ + q * C::kQBytes, pre_q[q][u], q0 + q * BM + 64 * half + lane + 32 * u < N,
+                         64 * half + lane + 32 * u, d);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[Bar::qfull()]);
+      for (int t = 0; t < T; ++t, ++g) {
+        const int st = g % S;
+        const uint4 cb[2] = {nb[0], nb[1]};
+        // Sign rows of the next K block: this item's next block, or block 0 of the next item.
+        {
+          int64_t nbh = bh;
+          int nt = t + 1;
+          bool any = true;
+          if (nt == T) {
+            nt = 0;
+            if (it + 1 < n_items) {
+              int nq0;
+              item_at(by_head, it + 1, p.H, nqb, BM * NQ, nbh, nq0);
+            } else {
+              any = false;
+            }
+          }
+          const uint4* nrows = reinterpret_cast<const uint4*>(p.bits_k) + nbh * N;
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int row = nt * BN + 64 * half + lane + 32 * u;
+            nb[u] = (any && row < N) ? __ldg(nrows + row) : zero4;
+          }
+        }
+        if (g >= S && !wait_warp(&bars[Bar::kvempty(st)], ((g / S) - 1) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int r = 64 * half + lane + 32 * u;
+          expand_row<DQ>(sK + st * C::kKBytes, cb[u], t * BN + r < N, r, d);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[Bar::kvfull(st)]);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    // Per block n (counted across items): P.V of block n-1 first (it needs no new operands),
+    // then QK of block n into the same S columns (issue order keeps P read before S is
+    // rewritten). The first P.V of an item starts the tile's other accumulator, so the previous
+    // item's epilogue can still read the one it ended in.
+    if (lane == 0) {
+      const uint32_t idesc_qk = (1u << 4) | (0u << 7) | (0u << 10) | (static_cast<uint32_t>(BN >> 3) << 17) |
+                                (static_cast<uint32_t>(BM >> 4) << 24);
+      const uint32_t idesc_pv = (2u << 4) | (0u << 7) | (1u << 10) | (1u << 16) |
+                                (static_cast<uint32_t>(DP >> 3) << 17) | (static_cast<uint32_t>(BM >> 4) << 24);
+      bool ok = true;
+      uint32_t cur_acc = (1u << NQ) - 1u;  // bit q: the accumulator P.V of tile q adds into
+      const int nblocks = n_items * T;
+      // Step n: P.V of block n - 1 (if n > 0), then QK of block n (if n < nblocks); t is the
+      // item-relative index of block n.
+      for (int n = 0, it = 0, t = 0; n <= nblocks && ok; ++n) {
+        if (n < nblocks && t == 0) {
+          if (!wait_bounded(&bars[Bar::qfull()], it & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+        }
+        const int tp = (t == 0 ? T : t) - 1;  // item-relative index of block n - 1
+        for (int q = 0; q < NQ && ok; ++q) {
+          if (n > 0) {
+            if (!wait_bounded(&bars[Bar::pfull(q)], (n - 1) & 1, abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            // Switch to the other accumulator (overwriting it) at an item's first block and
+            // when a row of the tile raised its max: the softmax warps' votes, written before
+            // their p_full arrivals.
+            bool fresh = tp == 0;
+            if (!fresh) {
+              const volatile uint32_t* vt = votes + (((n - 1) & 1) * NQ + q) * 4;
+              fresh = (vt[0] | vt[1] | vt[2] | vt[3]) != 0u;
+            }
+            if (fresh) cur_acc ^= 1u << q;
+            const uint32_t acc = tmem + C::tO(q, (cur_acc >> q) & 1u);
+            const uint32_t vbase = smem_u32(sV + ((n - 1) % S) * C::kVBytes);
+#pragma unroll
+            for (int kk = 0; kk < BN / 32; ++kk)
+              mma_i8_ts(acc, tmem + C::tP(q) + 8 * kk, smem_desc(vbase + 512 * kk, 128, 2048), idesc_pv,
+                        (fresh && kk == 0) ? 0u : 1u);
+            if (tp == T - 1) tc_commit(&bars[Bar::odone(q)]);
+          }
+          if (n < nblocks) {
+            if (q == 0) {
+              if (!wait_bounded(&bars[Bar::kvfull(n % S)], (n / S) & 1, abort_flag)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+            }
+            const uint32_t qb = smem_u32(sQ + q * C::kQBytes), kb = smem_u32(sK + (n % S) * C::kKBytes);
+#pragma unroll
+            for (int kk = 0; kk < DQ / 32; ++kk)
+              mma_f8f6f4_ss(tmem + C::tS(q), smem_desc(qb + kk * 4096, 2048, 128),
+                            smem_desc(kb + kk * 4096, 2048, 128), idesc_qk, kk > 0 ? 1u : 0u);
+            tc_commit(&bars[Bar::sfull(q)]);
+          }
+        }
+        if (!ok) break;
+        if (n > 0) tc_commit(&bars[Bar::kvempty((n - 1) % S)]);
+        // The item's Q tiles are free once its last QKs have read them.
+        if (n < nblocks && t == T - 1) tc_commit(&bars[Bar::qempty()]);
+        if (++t == T) {
+          t = 0;
+          ++it;
+        }
+      }
+      // Every MMA this thread issued has completed before tensor memory is released.
+      tc_commit(&bars[Bar::drain()]);
+      wait_bounded(&bars[Bar::drain()], 0, abort_flag, false);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ softmax warpgroups
+    const int q = (warp - 4) >> 2, w4 = warp & 3;
+    const int r = w4 * 32 + lane;
+    const uint32_t lane_base = static_cast<uint32_t>(w4 * 32) << 16;
+    const uint32_t aS = tmem + lane_base + C::tS(q);
+    const uint32_t aP = tmem + lane_base + C::tP(q);
+    const uint32_t aO0 = tmem + lane_base + C::tO(q, 0);
+    const uint32_t aO1 = tmem + lane_base + C::tO(q, 1);
+    const uint32_t aF = tmem + lane_base + C::tF(q);  // unused when F is in shared memory
+    // Fast path: full key blocks, no debug output, aligned dense rows, rel-pos table in shared
+    // memory with the class tokens handled by the zero padding.
+    const bool fast_ok = (p.dbg_logits == nullptr) &&
+                         (BK != BA_BIAS_DENSE || ((N & 3) == 0 && (p.bias.batch_stride & 3) == 0)) &&
+                         (!is_relpos(BK) || p.bias.n_prefix == 0 || tab_mode == 2);
+    bool alive = true;
+    // Accumulator that P.V of the current block adds into (tile-uniform): every item starts on
+    // the other one, as the MMA thread does.
+    int cur = 1;
+    float mu_q_next = 0.0f, mu_k_next = 0.0f;  // mu of the item about to start (loaded one item ahead)
+    int n0 = 0;  // index, counted across items, of the item's first key block
+    for (int it = 0; it < n_items && alive; ++it, n0 += T) {
+    int64_t bh;
+    int q0;
+    item_at(by_head, it, p.H, nqb, BM * NQ, bh, q0);
+    const int64_t b = bh / p.H, h = bh - b * p.H;
+    const int i = q0 + q * BM + r;
+    const bool row_ok = i < N;
+    const int ic = row_ok ? i : N - 1;  // rows past N read the bias of row N-1 (never stored)
+    if (it == 0) {
+      mu_q_next = p.mu_q[bh];
+      mu_k_next = p.mu_k[bh];
+    }
+    const float alpha = __fmul_rn(__fmul_rn(p.softmax_scale, mu_q_next), mu_k_next);
+    const float2 alpha2 = make_float2(alpha, alpha);
+
+    // Bias addressing. Dense: this row of [H][N][N]. Rel-pos: b_ij = tab[a_i - koff_j] with
+    // tab the head's table (staged in shared memory when it fits, followed by zeros that
+    // class-token rows and keys index into), koff_j kept as byte offsets.
+    const float* brow = nullptr;
+    const float* gtab = nullptr;
+    int a_i = 0;
+    if (BK == BA_BIAS_DENSE) brow = p.bias.data + b * p.bias.batch_stride + (h * N + ic) * N;
+    if (is_relpos(BK)) {
+      const int W2 = 2 * p.bias.table_w - 1;
+      gtab = p.bias.data + h * static_cast<int64_t>(2 * p.bias.table_h - 1) * W2;
+      if (ic >= p.bias.n_prefix) {
+        const int ti = ic - p.bias.n_prefix;
+        const int yi = ti / p.bias.grid_w;
+        a_i = (yi + p.bias.table_h - 1) * W2 + (ti - yi * p.bias.grid_w) + p.bias.table_w - 1;
+      } else {
+        a_i = (tab_mode == 2) ? tsize + kmax : -1;  // class-token row: the zeros (or the general path)
+      }
+    }
+    const uint32_t tb = smem_u32(stab) + 4u * static_cast<uint32_t>(a_i);  // this row's table base
+    const float* grow = gtab + a_i;  // this row's base in a table left in global memory
+
+    float m = -CUDART_INF_F, l = 0.0f;
+    // Whether F holds anything yet, and how many blocks the current accumulator holds.
+    int nblk = 1;
+    bool f_valid = false;
+    cur ^= 1;
+
+    for (int t = 0; t < T && alive; ++t) {
+      const int n = n0 + t;
+      const int st = n % S;
+      const int nk = min(BN, N - t * BN);
+      // 32-key chunks that hold keys of this block. The P codes of the chunks past them are
+      // left as they are: they multiply V rows past N, which the V copy fills with zeros.
+      const int nch = (nk + 31) >> 5;
+      if (is_relpos(BK) && !wait_warp(&bars[Bar::kvfull(st)], (n / S) & 1, abort_flag)) {
+        alive = false;
+        break;
+      }
+      if (!wait_warp(&bars[Bar::sfull(q)], n & 1, abort_flag)) {
+        alive = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t ko_s = smem_u32(koff + st * BN);
+
+      // Pass 1: s = alpha * x + b written back over S in TMEM; block max. The next 32-column
+      // block is loaded from TMEM while this one is computed.
+      float mx[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
+      // The fast path also takes a partial last block (keys past N are masked to -inf after
+      // the fact; their rel-pos offsets point at valid entries), except for dense bias rows,
+      // which end at N.
+      const bool fast = fast_ok && (nk == BN || BK != BA_BIAS_DENSE);
+      {
+        // One copy of the block body (a small hot loop stays in the instruction cache; the
+        // other softmax warps of the SM cover the TMEM load latency).
+#pragma unroll 1
+        for (int c = 0; c < nch; ++c) {
+          uint32_t x[32];
+          tmem_ld32(aS + 32 * c, x);
+          tmem_ld_wait();
+          reg_fence32(x);
+          if (fast) {
+            if (nk == BN)
+              fast_block<BK, false>(x, c, nk, alpha2, brow + t * BN, ko_s, tb, grow, tab_mode, mx);
+            else
+              fast_block<BK, true>(x, c, nk, alpha2, brow + t * BN, ko_s, tb, grow, tab_mode, mx);
+          } else {
+            // General path: a partial last block, class tokens without zero padding,
+            // unaligned dense rows, a table in global memory, or the debug logits.
+#pragma unroll
+            for (int u = 0; u < 32; ++u) {
+              const int j = 32 * c + u;
+              float sv = -CUDART_INF_F;
+              if (j < nk) {
+                const float xf = __uint_as_float(x[u]);
+                float bias = 0.0f;
+                if (BK == BA_BIAS_DENSE) bias = __ldg(brow + t * BN + j);
+                if (is_relpos(BK)) {
+                  const int kj = lds_s32(ko_s + 4u * j) >> 2;
+                  if (a_i >= 0 && kj >= 0)
+                    bias = (tab_mode != 0) ? lds_f32(smem_u32(stab) + 4u * static_cast<uint32_t>(a_i - kj))
+                                           : __ldg(gtab + (a_i - kj));
+                }
+                sv = __fmaf_rn(alpha, xf, bias);
+                if (p.dbg_logits != nullptr && row_ok)
+                  p.dbg_logits[(bh * N + i) * N + t * BN + j] = __float2int_rn(xf);
+              }
+              mx[u & 3] = fmaxf(mx[u & 3], sv);
+              x[u] = __float_as_uint(sv);
+            }
+          }
+          tmem_st32(aS + 32 * c, x);
+        }
+      }
+      const float m_new = fmaxf(m, fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])));
+      tmem_st_wait();
+
+      // Pass 2: P~ = 2^((s - m) log2 e) (masked keys hold s = -inf: P~ = 0), row sum, u8 codes
+      // -> TMEM columns 0..31 (their s values were read in the first step of this pass).
+      const float2 negm2 = make_float2(-m_new, -m_new);
+      const float2 log2e2 = make_float2(kLog2e, kLog2e);
+      const float2 c255 = make_float2(255.0f, 255.0f);
+      const float2 magic2 = make_float2(12582912.0f, 12582912.0f);
+      float2 lt2[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
+      {
+#pragma unroll 1
+        for (int c = 0; c < nch; ++c) {
+          uint32_t x[32];
+          tmem_ld32(aS + 32 * c, x);
+          tmem_ld_wait();
+          reg_fence32(x);
+          uint32_t pk[8];
+#pragma unroll
+          for (int w = 0; w < 8; ++w) {
+            uint32_t y[4];
+#pragma unroll
+            for (int e2 = 0; e2 < 2; ++e2) {
+              const int u = 4 * w + 2 * e2;
+              // s - m first (exact near the max), then the scale to base 2.
+              const float2 t2 = __fmul2_rn(
+                  __fadd2_rn(make_float2(__uint_as_float(x[u]), __uint_as_float(x[u + 1])), negm2), log2e2);
+              const float2 p2 = ((kPolyPairs >> (2 * w + e2)) & 1u) ? exp2_poly2(t2)
+                                                                    : make_float2(ex2_approx(t2.x), ex2_approx(t2.y));
+              lt2[e2] = __fadd2_rn(lt2[e2], p2);
+              // 255 P~ + 1.5 * 2^23: one rounding to the nearest integer (ties to even); the
+              // integer sits in the low byte of the result (P~ <= 1).
+              const float2 y2 = __ffma2_rn(p2, c255, magic2);
+              y[2 * e2] = __float_as_uint(y2.x);
+              y[2 * e2 + 1] = __float_as_uint(y2.y);
+            }
+            pk[w] = __byte_perm(__byte_perm(y[0], y[1], 0x0040), __byte_perm(y[2], y[3], 0x0040), 0x5410);
+          }
+          tmem_st8(aP + 8 * c, pk);
+        }
+      }
+      const float lt = (lt2[0].x + lt2[0].y) + (lt2[1].x + lt2[1].y);
+      // Rescale factor of the row's earlier blocks: exactly 1 while its max is unchanged.
+      const float ct = (m == -CUDART_INF_F) ? 0.0f : (m_new > m ? ex2_approx((m - m_new) * kLog2e) : 1.0f);
+      l = l * ct + lt;
+      // Vote (per warp) whether a row raised its max; the MMA thread reads the votes of the
+      // tile's four warps after their p_full arrivals.
+      const bool rose = __any_sync(0xffffffffu, t > 0 && m_new > m);
+      if (lane == 0) votes[((n & 1) * NQ + q) * 4 + w4] = rose ? 1u : 0u;
+      m = m_new;
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[Bar::pfull(q)]);
+      if (t == 0) continue;
+      // While the MMAs of the next block run: if any row of the tile raised its max, P.V of
+      // this block goes to the other accumulator, and the old one is folded into F with this
+      // row's factor (1 for rows whose max did not rise).
+      if (!wait_warp(&bars[Bar::pfull(q)], n & 1, abort_flag)) {
+        alive = false;
+        break;
+      }
+      const volatile uint32_t* vt = votes + ((n & 1) * NQ + q) * 4;
+      if ((vt[0] | vt[1] | vt[2] | vt[3]) != 0u) {
+        fold_rest<C, 0>(cur ? aO1 : aO0, aF, sF + q * BM + r, make_float2(ct, ct), !f_valid, nblk == 1);
+        if (!C::kFSmem) tmem_st_wait();
+        cur ^= 1;
+        f_valid = true;
+        nblk = 1;
+      } else {
+        ++nblk;
+      }
+    }
+
+    // This item's V scales / 255 (lane l of every warp holds channels l, l + 32, ..., read by
+    // shuffles in the epilogue) and the next item's mu, loaded while the last P.V runs.
+    float scv[(DP + 31) / 32];
+#pragma unroll
+    for (int k = 0; k < (DP + 31) / 32; ++k)
+      scv[k] = (32 * k + lane < d) ? p.v_scale[bh * d + 32 * k + lane] * (1.0f / 255.0f) : 0.0f;
+    if (it + 1 < n_items) {
+      int64_t nbh;
+      int nq0;
+      item_at(by_head, it + 1, p.H, nqb, BM * NQ, nbh, nq0);
+      mu_q_next = p.mu_q[nbh];
+      mu_k_next = p.mu_k[nbh];
+    }
+    if (alive && wait_warp(&bars[Bar::odone(q)], it & 1, abort_flag)) {
+      tc_fence_after();
+      const float inv_l = 1.0f / l;
+      // Rows whose byte length is a multiple of 16 are written with 16-byte stores (each
+      // thread owns one row); other shapes fall back to element stores.
+      const int esz = (p.o_dt == BA_F32) ? 4 : 2;
+      const bool vec = ((d * esz) & 15) == 0;
+      char* orow = reinterpret_cast<char*>(p.o) + ((bh * N + i) * d) * esz;
+      const uint32_t aO = cur ? aO1 : aO0;
+      const float4* fr = sF + q * BM + r;
+#pragma unroll 1
+      for (int cc = 0; cc < DP / 16; ++cc) {
+        uint32_t a[16], fb[16];
+        tmem_ld16(aO + 16 * cc, a);
+        if constexpr (!C::kFSmem) tmem_ld16(aF + 16 * cc, fb);  // read even before the first fold
+        tmem_ld_wait();
+        reg_fence16(a);
+        if constexpr (!C::kFSmem) reg_fence16(fb);
+        float val[16];
+        // Scales of channels 16 cc .. 16 cc + 15: held by lanes 16 (cc & 1) ... of register cc / 2.
+        float sreg = scv[0];
+#pragma unroll
+        for (int k = 1; k < (DP + 31) / 32; ++k)
+          if (cc >= 2 * k) sreg = scv[k];  // constant comparisons keep scv in registers
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          float fv;
+          if constexpr (C::kFSmem) {
+            const float4 v4 = fr[(4 * cc + (e >> 2)) * (NQ * BM)];
+            fv = (e & 3) == 0 ? v4.x : ((e & 3) == 1 ? v4.y : ((e & 3) == 2 ? v4.z : v4.w));
+          } else {
+            fv = __uint_as_float(fb[e]);
+          }
+          if (!f_valid) fv = 0.0f;
+          const float sc = __shfl_sync(0xffffffffu, sreg, 16 * (cc & 1) + e);
+          val[e] = (fv + __int2float_rn(static_cast<int>(a[e]))) * sc * inv_l;
+        }
+        if (!row_ok) continue;
+        if (vec && 16 * cc + 16 <= d) {
+          if (p.o_dt == BA_F32) {
+#pragma unroll
+            for (int k4 = 0; k4 < 4; ++k4)
+              reinterpret_cast<float4*>(orow + (16 * cc + 4 * k4) * 4)[0] =
+                  make_float4(val[4 * k4], val[4 * k4 + 1], val[4 * k4 + 2], val[4 * k4 + 3]);
+          } else {
+            uint32_t h[8];
+#pragma unroll
+            for (int k2 = 0; k2 < 8; ++k2) {
+              if (p.o_dt == BA_F16) {
+                const __half2 v = __floats2half2_rn(val[2 * k2], val[2 * k2 + 1]);
+                h[k2] = *reinterpret_cast<const uint32_t*>(&v);
+              } else {
+                const __nv_bfloat162 v = __floats2bfloat162_rn(val[2 * k2], val[2 * k2 + 1]);
+                h[k2] = *reinterpret_cast<const uint32_t*>(&v);
+              }
+            }
+            reinterpret_cast<uint4*>(orow + 16 * cc * 2)[0] = make_uint4(h[0], h[1], h[2], h[3]);
+            reinterpret_cast<uint4*>(orow + 16 * cc * 2)[1] = make_uint4(h[4], h[5], h[6], h[7]);
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            if (16 * cc + e < d) store_out(p.o, (bh * N + i) * d + 16 * cc + e, val[e], p.o_dt);
+        }
+      }
+    }
+    }
+  }
+
+  // ------------------------------------------------------------ teardown
+  tc_fence_before();
+  named_barrier_sync(1, C::kThreads);
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+// The same forward with one work item per CTA (no persistent loop): used for heads wider than
+// 80 channels (one 128-row tile per CTA, F in tensor memory), where it measured faster than the
+// persistent kernel on B200.
+template <int DP, int BK, int NQ_>
+__global__ void __launch_bounds__(Cfg<DP, NQ_>::kThreads, Cfg<DP, NQ_>::kCtasPerSm)
+    attn_tc_single_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmap_v, int tab_mode, int tsize,
                    int kmax) {
   using C = Cfg<DP, NQ_>;
   constexpr int NQ = C::NQ, DQ = C::DQ, S = C::kStages;
@@ -858,6 +1476,14 @@ int relpos_table_mode(const AttnParams& p) {
 }
 
 template <int DP, int BK, int NQ>
+constexpr auto pick_kernel() {
+  if constexpr (DP > 80)
+    return attn_tc_single_kernel<DP, BK, NQ>;
+  else
+    return attn_tc_kernel<DP, BK, NQ>;
+}
+
+template <int DP, int BK, int NQ>
 cudaError_t launch_cfg(const AttnParams& p, const CUtensorMap& tm, cudaStream_t s) {
   using C = Cfg<DP, NQ>;
   int tab_mode = 0, tsize = 0, kmax = 0;
@@ -872,17 +1498,35 @@ cudaError_t launch_cfg(const AttnParams& p, const CUtensorMap& tm, cudaStream_t 
   int smem = C::kTabOff + tab_bytes + 1024;
   const int floor_bytes = C::kCtasPerSm == 1 ? 116 * 1024 : 80 * 1024;
   if (smem < floor_bytes) smem = floor_bytes;
+  // Heads wider than 80 channels: one work item per CTA; otherwise the persistent kernel.
+  constexpr bool kSingle = DP > 80;
+  auto kernel = pick_kernel<DP, BK, NQ>();
   static int configured = 0;
   if (smem > configured) {
-    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<DP, BK, NQ>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(attn_tc_kernel<DP, BK, NQ>, cudaFuncAttributePreferredSharedMemoryCarveout,
-                             cudaSharedmemCarveoutMaxShared);
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
     configured = smem;
   }
-  const int64_t grid = static_cast<int64_t>(p.B) * p.H * ceil_div(p.N, BM * C::NQ);
-  attn_tc_kernel<DP, BK, NQ><<<static_cast<unsigned>(grid), C::kThreads, smem, s>>>(p, tm, tab_mode, tsize, kmax);
+  // Persistent CTAs: as many as fit at once (CTAs per SM x SMs), H per group, each walking the
+  // items of its head; at least one CTA per head.
+  int dev = 0, sms = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  const int64_t per_head = static_cast<int64_t>(p.B) * ceil_div(p.N, BM * C::NQ);
+  const int64_t slots = static_cast<int64_t>(C::kCtasPerSm) * sms;
+  int64_t grid;
+  if (kSingle) {
+    grid = per_head * p.H;
+  } else if (is_relpos(BK) && tab_mode != 0) {  // items grouped by head (the kernel's by_head)
+    const int64_t k = std::max<int64_t>(1, std::min<int64_t>(per_head, slots / p.H));
+    grid = k * p.H;
+  } else {
+    grid = std::min<int64_t>(per_head * p.H, slots);
+  }
+  kernel<<<static_cast<unsigned>(grid), C::kThreads, smem, s>>>(p, tm, tab_mode, tsize, kmax);
   return cudaGetLastError();
 }
 
