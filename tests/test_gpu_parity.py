@@ -115,6 +115,10 @@ EDGE = [  # B, H, N, d, dtype, bias kind, extra
     (1, 1, 300, 128, "bf16", 0, {}), (2, 3, 255, 64, "f16", 2, {"grid": (2, 127), "n_prefix": 1}),
     (1, 2, 256, 96, "bf16", 1, {"batch_bias": True}), (2, 2, 128, 16, "f16", 1, {}),
     (1, 1, 384, 8, "bf16", 0, {}), (1, 2, 200, 100, "f16", 1, {}), (3, 1, 513, 64, "bf16", 1, {"batch_bias": True}),
+    # persistent CTAs: more heads than CTAs fit at once (one CTA per head, several waves), and
+    # many items per CTA over ragged sequences (items grouped by head / spread over all CTAs)
+    (2, 300, 70, 32, "f16", 2, {"grid": (7, 10)}), (40, 12, 150, 64, "bf16", 2, {"grid": (10, 15)}),
+    (24, 16, 90, 48, "f16", 1, {}),
 ]
 
 
@@ -127,7 +131,10 @@ def test_edge_shapes(ba, case, impl):
     dtype = torch.float16 if dt == "f16" else torch.bfloat16
     w = inputs.random_case(B, H, N, d, dtype, kind, seed=N * 7 + d, **extra)
     out, lg = _forward(ba, w, impl, debug_logits=True)
-    assert_o_close(out.cpu().numpy(), oracle_forward(w), f"edge {case}")
+    want = oracle_forward(w)
+    assert_o_close(out.cpu().numpy(), want, f"edge {case}")
+    # without the debug output the kernels take their fast paths
+    assert_o_close(_forward(ba, w, impl).cpu().numpy(), want, f"edge {case} (fast path)")
     o = oracle.get()
     q, k, _ = oracle_qkv(w)
     assert np.array_equal(lg.cpu().numpy(), o.logits(o.pack_signs(q), o.pack_signs(k), d))
