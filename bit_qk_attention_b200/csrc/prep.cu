@@ -15,6 +15,8 @@
 // 16-byte pieces of consecutive rows), many in flight per thread. The |x| sums are taken in
 // double, where every partial sum of 16-bit magnitudes is exact, so they do not depend on the
 // summation order.
+#include <type_traits>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -257,6 +259,50 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(QuantParams p) {
   }
 }
 
+// 16-byte pieces of eight 16-bit values: the sign byte (bit e = x_e < 0 by IEEE compare: -0.0 and
+// NaN give 0) and the double sum of |x| (each magnitude exact in double; every partial sum
+// exact, so the order is free). fp16 works on the packed halves: a half2 compare gives a lane
+// mask per word, and each magnitude (sign bit cleared) converts straight to double.
+__device__ __forceinline__ double f16_to_f64(uint32_t bits16) {
+  double r;
+  const unsigned short h = static_cast<unsigned short>(bits16);
+  asm("cvt.f64.f16 %0, %1;" : "=d"(r) : "h"(h));
+  return r;
+}
+
+template <typename T>
+__device__ __forceinline__ uint32_t piece_sign_abs(const uint4& u, double& acc) {
+  if constexpr (std::is_same<T, __half>::value) {
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    uint32_t x = 0;
+    double a8[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      __half2 h2;
+      *reinterpret_cast<uint32_t*>(&h2) = w[i];
+      const uint32_t m = __hlt2_mask(h2, __float2half2_rn(0.0f));  // 0xFFFF per lane below zero
+      x |= (m & 0x00010001u) << (2 * i);  // element 2i at bit 2i, element 2i + 1 at bit 16 + 2i
+      const uint32_t a = w[i] & 0x7FFF7FFFu;
+      a8[2 * i] = f16_to_f64(a & 0xFFFFu);
+      a8[2 * i + 1] = f16_to_f64(a >> 16);
+    }
+    acc += ((a8[0] + a8[1]) + (a8[2] + a8[3])) + ((a8[4] + a8[5]) + (a8[6] + a8[7]));
+    return (x | (x >> 15)) & 0xFFu;
+  } else {
+    float f[8];
+    unpack8<T>(u, f);
+    uint32_t byte = 0;
+    double a8[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      byte |= (f[e] < 0.0f ? 1u : 0u) << e;
+      a8[e] = static_cast<double>(fabsf(f[e]));
+    }
+    acc += ((a8[0] + a8[1]) + (a8[2] + a8[3])) + ((a8[4] + a8[5]) + (a8[6] + a8[7]));
+    return byte;
+  }
+}
+
 // ---------------------------------------------------------------------------------------
 // Warp-granular streaming for rows of whole 16-byte pieces (d % 8 == 0). A warp covers
 // rpp = 32 / (d/8) rows per pass, lane (row-in-pass, piece) reading one 16-byte piece, so a
@@ -426,7 +472,9 @@ __global__ void __launch_bounds__(kThreads, 3) prep_slice_kernel(SliceParams p) 
   __shared__ double sred[kThreads / 32];
   const PrepDims& g = p.g;
   const int64_t bh = blockIdx.x;
-  const int job = blockIdx.y;  // 0: q, 1: k, 2: v
+  // 0: q, 1: k, 2: v. The v CTAs (two passes over their slice) are the longest: they take the
+  // first grid row, so they are scheduled first and the q and k CTAs fill in behind them.
+  const int job = (static_cast<int>(blockIdx.y) + 2) % 3;
   const int d = g.d, dp = g.dp;
   const int tpr = d >> 3;
   const int rpp = kThreads / tpr;
@@ -452,20 +500,7 @@ __global__ void __launch_bounds__(kThreads, 3) prep_slice_kernel(SliceParams p) 
 #pragma unroll
       for (int j = 0; j < kSliceBatch; ++j) {
         const int r = j * rpp + rp;
-        if (on && r < nrow) {
-          float f[8];
-          unpack8<T>(u[j], f);
-          uint32_t byte = 0;
-          double a8[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            byte |= (f[e] < 0.0f ? 1u : 0u) << e;
-            a8[e] = static_cast<double>(fabsf(f[e]));
-          }
-          // Every partial sum of 16-bit magnitudes is exact in double: the order is free.
-          acc += ((a8[0] + a8[1]) + (a8[2] + a8[3])) + ((a8[4] + a8[5]) + (a8[6] + a8[7]));
-          sbits[r][sub] = static_cast<uint8_t>(byte);
-        }
+        if (on && r < nrow) sbits[r][sub] = static_cast<uint8_t>(piece_sign_abs<T>(u[j], acc));
       }
       __syncthreads();
       for (int r = threadIdx.x; r < nrow; r += kThreads) bits[r0 + r] = *reinterpret_cast<const uint4*>(sbits[r]);
@@ -475,10 +510,11 @@ __global__ void __launch_bounds__(kThreads, 3) prep_slice_kernel(SliceParams p) 
     if (threadIdx.x == 0) (job == 0 ? p.mu_q : p.mu_k)[bh] = static_cast<float>(tot / (static_cast<double>(g.N) * d));
     return;
   }
-  // v: channel maxima over the slice.
+  // v: channel maxima over the slice (fp16: packed half2 maxima of the magnitudes, exact).
   float mx[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) mx[e] = 0.0f;
+  uint32_t hm[4] = {0u, 0u, 0u, 0u};  // fp16: |v| maxima as half2 bit patterns (0 = +0.0)
   for (int r0 = 0; r0 < g.N; r0 += rows_per_batch) {
     const int nrow = min(rows_per_batch, g.N - r0);
     uint4 u[kSliceBatch];
@@ -491,12 +527,28 @@ __global__ void __launch_bounds__(kThreads, 3) prep_slice_kernel(SliceParams p) 
     for (int j = 0; j < kSliceBatch; ++j) {
       const int r = j * rpp + rp;
       if (on && r < nrow) {
-        float f[8];
-        unpack8<T>(u[j], f);
+        if constexpr (std::is_same<T, __half>::value) {
+          const uint32_t w[4] = {u[j].x, u[j].y, u[j].z, u[j].w};
 #pragma unroll
-        for (int e = 0; e < 8; ++e) mx[e] = fmaxf(mx[e], fabsf(f[e]));
+          for (int i = 0; i < 4; ++i) {
+            __half2 a, b;
+            *reinterpret_cast<uint32_t*>(&a) = w[i] & 0x7FFF7FFFu;
+            *reinterpret_cast<uint32_t*>(&b) = hm[i];
+            const __half2 c = __hmax2(a, b);
+            hm[i] = *reinterpret_cast<const uint32_t*>(&c);
+          }
+        } else {
+          float f[8];
+          unpack8<T>(u[j], f);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) mx[e] = fmaxf(mx[e], fabsf(f[e]));
+        }
       }
     }
+  }
+  if constexpr (std::is_same<T, __half>::value) {
+    const uint4 hv = make_uint4(hm[0], hm[1], hm[2], hm[3]);
+    unpack8<T>(hv, mx);
   }
   __shared__ float sinv[128];
   if (on) {
