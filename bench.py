@@ -125,6 +125,22 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
+def max_over_ranks(ms: float, dist, device) -> float:
+    """The job's time: the largest of the ranks' device times (all ranks take part)."""
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(ops: float, tokens: float, ms_per_step: float, world: int):
+    """Whole-job effective TOPS and tokens/s: every rank runs the same step on its own replica
+    of the workload (weak scaling), so the job does world times the work in the slowest rank's
+    time."""
+    sec = ms_per_step / 1e3
+    return world * ops / sec / 1e12, world * tokens / sec
+
+
 def dist_info():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -268,12 +284,9 @@ def main():
     clk = clocks.stop()
     ms = e0.elapsed_time(e1)
     if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+        ms = max_over_ranks(ms, dist, dev)
     ms_per_step = ms / args.steps
-    value = world * ops / (ms_per_step / 1e3) / 1e12
-    tok_s = world * tokens / (ms_per_step / 1e3)
+    value, tok_s = job_throughput(ops, tokens, ms_per_step, world)
     ba.check_device_status()
 
     # Per-stage device times (a separate pass with CUDA events around each kernel).
@@ -352,10 +365,8 @@ def main():
         torch.cuda.synchronize()
         e_ms = a0.elapsed_time(a1) / ne
         if world > 1:
-            t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
-        e2e = {"value": world * ops / (e_ms / 1e3) / 1e12, "unit": UNIT,
+            e_ms = max_over_ranks(e_ms, dist, dev)
+        e2e = {"value": job_throughput(ops, tokens, e_ms, world)[0], "unit": UNIT,
                "h2d_bytes_per_step": 3 * E * esz, "d2h_bytes_per_step": E * esz, "ms_per_step": e_ms}
 
     cpu = None
