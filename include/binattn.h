@@ -134,8 +134,9 @@ ba_status ba_attention_fwd_packed(const uint32_t* bits_q, const float* mu_q, con
                                   void* o, ba_dtype o_dt, int32_t* dbg_logits, void* stream);
 
 /*
- * The whole forward pass: ba_pack_signs(q), ba_pack_signs(k), ba_quant_v(v) into the
- * workspace, then ba_attention_fwd_packed.
+ * The whole forward pass: the results of ba_pack_signs(q), ba_pack_signs(k) and ba_quant_v(v)
+ * into the workspace (in one launch for the shapes ba_prep_fused reports, else three), then
+ * the fused step of ba_attention_fwd_packed.
  *   q, k, v: [B][H][N][d] in dt (BA_F16 or BA_BF16).
  *   ws:      at least ba_workspace_bytes(B,H,N,d) bytes; its contents on return are the
  *            packed operands (layout private to the library).
@@ -186,8 +187,9 @@ ba_status ba_check_device_status(void* stream);
 
 /*
  * Stage timing for measurement tools (off by default). While enabled, ba_attention_fwd
- * records a CUDA event on its stream before its first kernel and after each kernel: the
- * q/k/v streaming pass, the finalize pass, the V quantiser and the fused attention kernel.
+ * records a CUDA event on its stream before its first kernel and after each stage: the
+ * q/k/v streaming pass, the finalize pass, the V quantiser and the fused attention kernel
+ * (on the one-launch preparation path the finalize and quantiser stages are empty).
  * ba_stage_times synchronises on those events and writes the device time of each of the
  * four stages in milliseconds, summed over the calls since the last read, to ms[0..n-1]
  * (n <= 4), stores the number of calls in *calls, and forgets them.
