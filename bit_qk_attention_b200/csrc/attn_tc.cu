@@ -18,8 +18,8 @@
 //   * Warps 2 and 3 expand the 1-bit sign rows of Q (once) and of each K block into fp8 +-1
 //     operands in shared memory (channels >= d become 0); warp 0 TMA-loads the int8 V block
 //     (a 4-D tensor map that lands it in the MN-major core-matrix layout the MMA reads) and
-//     writes the block's rel-pos key offsets. A ring of 3 or 4 K/V stages decouples them
-//     from the MMAs.
+//     writes the block's rel-pos key offsets. A 4-stage ring of K/V blocks decouples them from
+//     the MMAs.
 //   * Warp 1 issues the MMAs from one thread:
 //       S  = Q . K^T   tcgen05.mma kind::f8f6f4 (e4m3 +-1, fp32 accumulate: exact integers)
 //       O += P . V     tcgen05.mma kind::i8, A = the uint8 codes read from TMEM, B = int8 V
