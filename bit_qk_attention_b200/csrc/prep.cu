@@ -205,15 +205,16 @@ __global__ void __launch_bounds__(128) finalize_kernel(FinalizeParams p) {
   }
 }
 
+// Four int8 codes rne(v * inv), packed. The product is rounded to fp32 first (as the definition
+// states), then to the nearest integer, ties to even, by adding 1.5 * 2^23: the integer lands in
+// the low mantissa bits, whose low byte is its two's-complement byte. The clamp to [-127, 127]
+// never acts on finite inputs: inv = rn(127 / amax) and |v| <= amax give
+// |rn(v * inv)| <= 127 (1 + 2^-24)^2 < 127.5.
 __device__ __forceinline__ uint32_t quant4(const float* f, const float* inv) {
-  uint32_t w = 0;
+  uint32_t y[4];
 #pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    int q = __float2int_rn(__fmul_rn(f[e], inv[e]));
-    q = max(-127, min(127, q));
-    w |= (static_cast<uint32_t>(q) & 0xffu) << (8 * e);
-  }
-  return w;
+  for (int e = 0; e < 4; ++e) y[e] = __float_as_uint(__fadd_rn(__fmul_rn(f[e], inv[e]), 12582912.0f));
+  return __byte_perm(__byte_perm(y[0], y[1], 0x0040), __byte_perm(y[2], y[3], 0x0040), 0x5410);
 }
 
 template <typename T>
@@ -262,12 +263,17 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(QuantParams p) {
 // 16-byte pieces of eight 16-bit values: the sign byte (bit e = x_e < 0 by IEEE compare: -0.0 and
 // NaN give 0) and the double sum of |x| (each magnitude exact in double; every partial sum
 // exact, so the order is free). fp16 works on the packed halves: a half2 compare gives a lane
-// mask per word, and each magnitude (sign bit cleared) converts straight to double.
-__device__ __forceinline__ double f16_to_f64(uint32_t bits16) {
-  double r;
-  const unsigned short h = static_cast<unsigned short>(bits16);
-  asm("cvt.f64.f16 %0, %1;" : "=d"(r) : "h"(h));
-  return r;
+// mask per word, and each magnitude is read as a double by bit placement alone (f16_scaled).
+//
+// An fp16 magnitude with exponent field e and fraction m, placed at bit 52 - 10 of a double
+// (fraction) and bit 52 (exponent field), is the double with exponent field e and fraction m:
+// (1 + m/2^10) 2^(e - 1023) for e >= 1 and m 2^-1032 for e = 0 (a subnormal double), i.e.
+// exactly |x| 2^-1008 in both cases. Sums of these scaled values round exactly as the sums of
+// |x| do (a power-of-two scale; below 2^-1022 every sum of multiples of 2^-1032 is exact), and
+// one multiply by 2^1008 at the end restores the scale.
+constexpr double kF16Unscale = 0x1p1008;
+__device__ __forceinline__ double f16_scaled(uint32_t hi_word) {
+  return __hiloint2double(static_cast<int>(hi_word), 0);
 }
 
 template <typename T>
@@ -283,8 +289,8 @@ __device__ __forceinline__ uint32_t piece_sign_abs(const uint4& u, double& acc) 
       const uint32_t m = __hlt2_mask(h2, __float2half2_rn(0.0f));  // 0xFFFF per lane below zero
       x |= (m & 0x00010001u) << (2 * i);  // element 2i at bit 2i, element 2i + 1 at bit 16 + 2i
       const uint32_t a = w[i] & 0x7FFF7FFFu;
-      a8[2 * i] = f16_to_f64(a & 0xFFFFu);
-      a8[2 * i + 1] = f16_to_f64(a >> 16);
+      a8[2 * i] = f16_scaled((a << 10) & 0x01FFFC00u);
+      a8[2 * i + 1] = f16_scaled((a >> 6) & 0x01FFFC00u);
     }
     acc += ((a8[0] + a8[1]) + (a8[2] + a8[3])) + ((a8[4] + a8[5]) + (a8[6] + a8[7]));
     return (x | (x >> 15)) & 0xFFu;
@@ -506,7 +512,8 @@ __global__ void __launch_bounds__(kThreads, 3) prep_slice_kernel(SliceParams p) 
       for (int r = threadIdx.x; r < nrow; r += kThreads) bits[r0 + r] = *reinterpret_cast<const uint4*>(sbits[r]);
       __syncthreads();
     }
-    const double tot = block_sum(acc, sred);
+    double tot = block_sum(acc, sred);
+    if constexpr (std::is_same<T, __half>::value) tot *= kF16Unscale;  // exact (see f16_scaled)
     if (threadIdx.x == 0) (job == 0 ? p.mu_q : p.mu_k)[bh] = static_cast<float>(tot / (static_cast<double>(g.N) * d));
     return;
   }

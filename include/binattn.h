@@ -98,7 +98,8 @@ size_t ba_workspace_bytes(int B, int H, int N, int d);
  *   x:    [B][H][N][d] in dt (BA_F16 or BA_BF16).
  *   bits: [B][H][N][4] uint32 out. Bit (c % 32) of word c/32 is 1 iff x_c < 0 (IEEE: -0.0,
  *         +0.0 and NaN give 0); bits at c >= d are 0.
- *   mu:   [B][H] fp32 out, mean of |x| over the N*d entries of each (b, h) slice.
+ *   mu:   [B][H] fp32 out, mean of |x| over the N*d entries of each (b, h) slice (x must be
+ *         finite: mu of a slice holding inf or NaN is unspecified).
  *   ws:   at least ba_pack_workspace_bytes(B,H,N,d) bytes of device memory (partial sums).
  */
 ba_status ba_pack_signs(const void* x, ba_dtype dt, int B, int H, int N, int d, uint32_t* bits,
@@ -108,7 +109,7 @@ ba_status ba_pack_signs(const void* x, ba_dtype dt, int B, int H, int N, int d, 
  * Channel-aware 8-bit V (gist.science/zh 2.2(3); gist.science/nl Methodologie 2: a
  * channel-specific scale). Per (b, h, c): amax = max_j |v_jc|, inv = 127/amax (fp32),
  * q = clamp(rne(v * inv), -127, 127), v_scale = amax/127; a zero channel gives q = 0 and
- * v_scale = 0.
+ * v_scale = 0. v must be finite (the codes of a channel holding inf or NaN are unspecified).
  *   v:       [B][H][N][d] in dt (BA_F16 or BA_BF16).
  *   vq:      [B][H][N][ba_v_row_bytes(d)] int8 out, pad columns 0.
  *   v_scale: [B][H][d] fp32 out.
