@@ -468,11 +468,16 @@ __global__ void __launch_bounds__(kThreads, 3) prep_warp_kernel(PrepParams p, in
 // passes of rpp = 256 / (d/8) rows (a slice of up to kSliceBatch * rpp rows in one batch, all of
 // its loads in flight at once), then reduces once: mu for q and k; for v the channel maxima, the
 // scales, and a second batch of loads (L2) that quantises. Sign bytes are assembled per batch
-// in shared memory and written as 16-byte rows.
+// in shared memory and written as 16-byte rows. Two batch depths: 7 passes when they hold the
+// slice in one batch (a DeiT-B slice, 197 rows of 64), which keeps the kernel within 64
+// registers so that four CTAs share an SM and more of one CTA's loads overlap another's
+// arithmetic; otherwise 10 passes at three CTAs per SM (the load slots past the slice's rows
+// cost issue slots, so the shallower batch is taken whenever it suffices).
+constexpr int kSliceBatchShort = 7;
 constexpr int kSliceBatch = 10;
 
-template <typename T>
-__global__ void __launch_bounds__(kThreads, 3) prep_slice_kernel(SliceParams p) {
+template <typename T, int kSliceBatch>
+__global__ void __launch_bounds__(kThreads, kSliceBatch <= kSliceBatchShort ? 4 : 3) prep_slice_kernel(SliceParams p) {
   __shared__ __align__(16) uint8_t sbits[kSliceBatch * kThreads / 4][16];  // d >= 32: at most 64 rows per pass
   __shared__ float smax[kThreads * 8];
   __shared__ double sred[kThreads / 32];
@@ -641,10 +646,18 @@ bool use_slice_prep(const PrepDims& g) {
 cudaError_t launch_prep_slices(const SliceParams& p, int dt, cudaStream_t s) {
   if ((p.g.d & 7) != 0 || p.g.d < 32) return cudaErrorInvalidValue;
   const dim3 grid(static_cast<unsigned>(p.g.BH), 3);
-  if (dt == BA_F16)
-    prep_slice_kernel<__half><<<grid, kThreads, 0, s>>>(p);
-  else
-    prep_slice_kernel<__nv_bfloat16><<<grid, kThreads, 0, s>>>(p);
+  const bool shallow = p.g.N <= kSliceBatchShort * (kThreads / (p.g.d >> 3));
+  if (dt == BA_F16) {
+    if (shallow)
+      prep_slice_kernel<__half, kSliceBatchShort><<<grid, kThreads, 0, s>>>(p);
+    else
+      prep_slice_kernel<__half, kSliceBatch><<<grid, kThreads, 0, s>>>(p);
+  } else {
+    if (shallow)
+      prep_slice_kernel<__nv_bfloat16, kSliceBatchShort><<<grid, kThreads, 0, s>>>(p);
+    else
+      prep_slice_kernel<__nv_bfloat16, kSliceBatch><<<grid, kThreads, 0, s>>>(p);
+  }
   return cudaGetLastError();
 }
 

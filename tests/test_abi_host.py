@@ -56,6 +56,8 @@ def test_host_queries(L):
     assert L.ba_prep_fused(1, 16, 4096, 64) == 0 and L.ba_prep_fused(64, 12, 197, 60) == 0
     assert L.ba_prep_fused(64, 12, 197, 16) == 0 and L.ba_prep_fused(0, 12, 197, 64) == 0
     assert L.ba_prep_fused(64, 12, 197, 129) == 0
+    # one launch while a slice fits in two batches of 10 passes: 2 * 10 * (256 / (d/8)) rows
+    assert L.ba_prep_fused(8, 16, 640, 64) == 1 and L.ba_prep_fused(8, 16, 641, 64) == 0
     assert L.ba_workspace_bytes(0, 4, 16, 64) == 0 and L.ba_workspace_bytes(2, 4, 0, 64) == 0
     big = L.ba_workspace_bytes(2, 16, 4096, 64)
     assert big >= 2 * 16 * 4096 * (16 + 16 + 64)

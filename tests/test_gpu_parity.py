@@ -119,6 +119,8 @@ EDGE = [  # B, H, N, d, dtype, bias kind, extra
     # many items per CTA over ragged sequences (items grouped by head / spread over all CTAs)
     (2, 300, 70, 32, "f16", 2, {"grid": (7, 10)}), (40, 12, 150, 64, "bf16", 2, {"grid": (10, 15)}),
     (24, 16, 90, 48, "f16", 1, {}),
+    # one-launch preparation with the deeper load batch (a slice longer than 7 passes of rows)
+    (16, 24, 300, 64, "bf16", 1, {}),
 ]
 
 
