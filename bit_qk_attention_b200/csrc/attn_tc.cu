@@ -418,6 +418,10 @@ __global__ void __launch_bounds__(Cfg<DP, NQ_>::kThreads, Cfg<DP, NQ_>::kCtasPer
     fence_proxy_async_smem();
     tma_prefetch_desc(&tmap_v);
   }
+  // Everything above reads only the caller's inputs; from here on the kernel reads the sign
+  // rows, mu and int8 V, which the preparation kernel before it in the stream may still be
+  // writing when this kernel was launched as its programmatic dependent.
+  grid_dependency_wait();
   // Warps 2 and 3 load the sign rows of their Q rows and of key block 0 of the first item
   // before the setup barrier, so the loads overlap the setup.
   const uint4 zero4 = make_uint4(0u, 0u, 0u, 0u);
@@ -1526,8 +1530,25 @@ cudaError_t launch_cfg(const AttnParams& p, const CUtensorMap& tm, cudaStream_t 
   } else {
     grid = std::min<int64_t>(per_head * p.H, slots);
   }
-  kernel<<<static_cast<unsigned>(grid), C::kThreads, smem, s>>>(p, tm, tab_mode, tsize, kmax);
-  return cudaGetLastError();
+  if constexpr (kSingle) {
+    kernel<<<static_cast<unsigned>(grid), C::kThreads, smem, s>>>(p, tm, tab_mode, tsize, kmax);
+    return cudaGetLastError();
+  } else {
+    // Programmatic dependent of the preparation kernel: the launch, and the barrier set-up of
+    // the CTAs that find an SM free, overlap the last preparation CTAs; each CTA waits for the
+    // preparation grid (grid_dependency_wait) before it reads anything that grid writes.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(C::kThreads);
+    cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, p, tm, tab_mode, tsize, kmax);
+  }
 }
 
 template <int DP, int NQ>

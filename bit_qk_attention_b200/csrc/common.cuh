@@ -62,6 +62,13 @@ __device__ __forceinline__ uint4 ldg_stream(const void* p) {
   return r;
 }
 
+// Programmatic dependent launch. A kernel launched with programmatic stream serialization may
+// start while the kernel before it in the stream is still running: grid_dependency_wait()
+// returns once that kernel has completed and its writes are visible (at once when there is no
+// such kernel). allow_dependents() lets the next kernel start before this one completes.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void allow_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // Output store of one fp32 value in the requested dtype.
 __device__ __forceinline__ void store_out(void* o, int64_t idx, float val, int o_dt) {
   if (o_dt == BA_F32) {

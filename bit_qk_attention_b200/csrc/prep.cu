@@ -219,6 +219,7 @@ __device__ __forceinline__ uint32_t quant4(const float* f, const float* inv) {
 
 template <typename T>
 __global__ void __launch_bounds__(kThreads) quant_kernel(QuantParams p) {
+  allow_dependents();  // the attention kernel may start early; it waits for this grid
   __shared__ float sinv[128];
   const int64_t cta = blockIdx.x;
   const int64_t bh = cta / p.g.nchunk;
@@ -478,6 +479,9 @@ constexpr int kSliceBatch = 10;
 
 template <typename T, int kSliceBatch>
 __global__ void __launch_bounds__(kThreads, kSliceBatch <= kSliceBatchShort ? 4 : 3) prep_slice_kernel(SliceParams p) {
+  // The attention kernel that follows may start on SMs this grid frees once every CTA of it
+  // is running; it waits for this grid's completion before it reads what this grid writes.
+  allow_dependents();
   __shared__ __align__(16) uint8_t sbits[kSliceBatch * kThreads / 4][16];  // d >= 32: at most 64 rows per pass
   __shared__ float smax[kThreads * 8];
   __shared__ double sred[kThreads / 32];
