@@ -181,6 +181,13 @@ __global__ void __launch_bounds__(kThreads) prep_kernel(PrepParams p) {
   }
 }
 
+// A channel gets codes when its maximum is nonzero and 127 / amax is a finite float. A bf16
+// channel with amax below 127 / FLT_MAX (about 3.7e-37) would get inv = +inf, codes of inf and
+// NaN: it is treated as a zero channel instead (codes 0, scale 0), as the definition reads.
+__device__ __forceinline__ bool channel_live(float amax, float inv) {
+  return amax > 0.0f && inv <= 3.402823466e38f;
+}
+
 __global__ void __launch_bounds__(128) finalize_kernel(FinalizeParams p) {
   const int64_t bh = blockIdx.x;
   const PrepDims& g = p.g;
@@ -198,8 +205,9 @@ __global__ void __launch_bounds__(128) finalize_kernel(FinalizeParams p) {
     for (int c = threadIdx.x; c < g.dp; c += blockDim.x) {
       float m = 0.0f;
       for (int ch = 0; ch < g.nchunk; ++ch) m = fmaxf(m, p.part_amax[(bh * g.nchunk + ch) * g.dp + c]);
-      const bool live = (c < g.d) && (m > 0.0f);
-      p.inv[bh * g.dp + c] = live ? __fdiv_rn(127.0f, m) : 0.0f;
+      const float inv = __fdiv_rn(127.0f, m);
+      const bool live = (c < g.d) && channel_live(m, inv);
+      p.inv[bh * g.dp + c] = live ? inv : 0.0f;
       if (c < g.d) p.v_scale[bh * g.d + c] = live ? __fdiv_rn(m, 127.0f) : 0.0f;
     }
   }
@@ -208,8 +216,8 @@ __global__ void __launch_bounds__(128) finalize_kernel(FinalizeParams p) {
 // Four int8 codes rne(v * inv), packed. The product is rounded to fp32 first (as the definition
 // states), then to the nearest integer, ties to even, by adding 1.5 * 2^23: the integer lands in
 // the low mantissa bits, whose low byte is its two's-complement byte. The clamp to [-127, 127]
-// never acts on finite inputs: inv = rn(127 / amax) and |v| <= amax give
-// |rn(v * inv)| <= 127 (1 + 2^-24)^2 < 127.5.
+// never acts on finite inputs: inv = rn(127 / amax) is finite (channel_live) and |v| <= amax
+// give |rn(v * inv)| <= 127 (1 + 2^-24)^2 < 127.5; a dead channel has inv = 0 and codes 0.
 __device__ __forceinline__ uint32_t quant4(const float* f, const float* inv) {
   uint32_t y[4];
 #pragma unroll
@@ -577,8 +585,9 @@ __global__ void __launch_bounds__(kThreads, kSliceBatch <= kSliceBatchShort ? 4 
     float m = 0.0f;
     if (c < d)
       for (int rr = 0; rr < rows; ++rr) m = fmaxf(m, smax[rr * d + c]);
-    const bool live = (c < d) && (m > 0.0f);
-    sinv[c] = live ? __fdiv_rn(127.0f, m) : 0.0f;
+    const float inv = __fdiv_rn(127.0f, m);
+    const bool live = (c < d) && channel_live(m, inv);
+    sinv[c] = live ? inv : 0.0f;
     if (c < d) p.v_scale[bh * d + c] = live ? __fdiv_rn(m, 127.0f) : 0.0f;
   }
   __syncthreads();

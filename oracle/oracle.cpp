@@ -115,6 +115,9 @@ void bao_logits(const uint32_t* bq, const uint32_t* bk, int64_t BH, int64_t N, i
 // tokens, range +-127, round to nearest even:
 //   amax_c = max_j |v_jc|;  inv = 127/amax_c (fp32);  q = clamp(rne(v*inv), -127, 127);
 //   sv_c = amax_c/127 (fp32). A zero channel gives q = 0 and sv_c = 0.
+// Reading for a channel so small that 127/amax_c overflows fp32 (amax_c < 127/FLT_MAX, only
+// reachable with bf16 inputs): inv is not a float there, so the channel is treated as a zero
+// channel (q = 0, sv_c = 0); its whole contribution to O is below 1e-36.
 // v: [BH][N][d], vq: [BH][N][d] int8, sv: [BH][d].
 void bao_quant_v(const float* v, int64_t BH, int64_t N, int d, int8_t* vq, float* sv) {
   for (int64_t s = 0; s < BH; ++s)
@@ -124,7 +127,7 @@ void bao_quant_v(const float* v, int64_t BH, int64_t N, int d, int8_t* vq, float
         const float a = std::fabs(v[(s * N + j) * d + c]);
         if (a > amax) amax = a;
       }
-      if (amax == 0.0f) {
+      if (amax == 0.0f || !std::isfinite(127.0f / amax)) {
         sv[s * d + c] = 0.0f;
         for (int64_t j = 0; j < N; ++j) vq[(s * N + j) * d + c] = 0;
         continue;

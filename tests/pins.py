@@ -144,6 +144,14 @@ def pin_quant_v_closed_forms(o: oracle_mod.Oracle):
     assert vq[0, 1, 0, 3] == -127 and vq[0, 1, N - 1, 3] == 127, "amax entries map to +-127"
     assert list(vq[0, 1, :, 4]) == [127, 2, 4, -2, -4, 0, 2, 0, 0], "round half to even"
     assert sv[0, 1, 4] == np.float32(1.0)
+    # A channel whose 127 / amax overflows fp32 (amax < 127 / FLT_MAX) is a zero channel; one
+    # just above that bound still maps its amax entries to +-127.
+    w = np.zeros((1, 1, 4, 2), np.float32)
+    w[0, 0, :, 0] = [1e-38, 0.0, -5e-39, 2e-39]
+    w[0, 0, :, 1] = [4e-37, 0.0, -4e-37, 2e-37]
+    wq, ws = o.quant_v(w)
+    assert np.all(wq[0, 0, :, 0] == 0) and ws[0, 0, 0] == 0.0, "overflowing 127/amax: zero channel"
+    assert list(wq[0, 0, :, 1]) == [127, 0, -127, 64] and ws[0, 0, 1] == np.float32(4e-37) / np.float32(127)
 
 
 def pin_quant_v_invariants(o: oracle_mod.Oracle):

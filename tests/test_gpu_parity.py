@@ -78,6 +78,37 @@ def test_quant_v(ba, name):
     assert np.array_equal(vs.cpu().numpy(), want_s), "V scales differ"
 
 
+@pytest.mark.parametrize("N", [197, 3000])  # one-launch slice path and the chunked path
+def test_quant_v_tiny_channels(ba, N):
+    """bf16 channels far below fp32's normal range: a channel whose 127 / amax overflows fp32 is a
+    zero channel (codes 0, scale 0), zeros inside a live tiny channel stay 0, and the amax entries
+    of a channel just above the bound map to +-127, bit-exact with the oracle."""
+    import torch
+    g = torch.Generator().manual_seed(N)
+    B, H, d = 64 if N == 197 else 2, 2, 64
+    v = torch.randn((B, H, N, d), generator=g)
+    v[:, :, :, 3] *= 1e-39   # 127 / amax overflows: a dead channel
+    v[:, :, ::5, 3] = 0.0
+    v[:, :, :, 7] *= 4e-37   # just above the bound
+    v[:, :, ::3, 7] = 0.0
+    v[:, :, :, 9] = 0.0
+    v = v.bfloat16()
+    vq, vs = ba.quant_v(v.cuda())
+    want_q, want_s = oracle.get().quant_v(v.float().numpy())
+    assert np.array_equal(vq.cpu().numpy()[..., :d], want_q), "V codes differ"
+    assert np.array_equal(vs.cpu().numpy(), want_s), "V scales differ"
+    assert np.all(want_q[:, :, :, 3] == 0) and np.all(want_s[:, :, 3] == 0)
+    assert np.abs(want_q[:, :, :, 7].astype(np.int32)).max() == 127
+    if N == 197:
+        assert ba.prep_fused(B, H, N, d)
+    # the whole step on the same v: O finite and within the bar
+    from bit_qk_attention_b200 import inputs
+    w = inputs.random_case(B, H, N, d, torch.bfloat16, 0, seed=N)
+    w.v = v
+    out = _forward(ba, w, 2).cpu().numpy()
+    assert_o_close(out, oracle_forward(w), "tiny channels")
+
+
 # ----------------------------------------------------------------------------- logits
 @pytest.mark.parametrize("impl", list(IMPLS.values()), ids=list(IMPLS))
 @pytest.mark.parametrize("name", ["tiny", "deit_b", "dit256"])
