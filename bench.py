@@ -3,11 +3,13 @@
 sign pack + mu, V quantiser, fused binary-QK / int8-PV attention) on synthetic inputs.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload deit_b|tiny|dit256|dit512|dit1024|sweep<N>_d<d>]
+                    [--workload sweep32768_d128|deit_b|tiny|dit256|dit512|dit1024|sweep<N>_d<d>]
 
-Prints ONE JSON line on rank 0. Under torchrun (N > 1) every rank runs the same workload on
-its own GPU (independent replicas: the path has no data-path exchange) and the time is the
-max over ranks.
+The default workload is the largest single-GPU configuration of the long-sequence sweep
+(B=1, H=16, N=32768, d=128, bf16, 2-D relative-position bias on a 128 x 256 grid); the
+others are there for measurement of the smaller shapes. Prints ONE JSON line on rank 0.
+Under torchrun (N > 1) every rank runs the same workload on its own GPU (independent
+replicas: the path has no data-path exchange) and the time is the max over ranks.
 """
 from __future__ import annotations
 
@@ -35,10 +37,10 @@ KERNEL_FILES = {"stream_qkv": "prep.cu", "finalize": "prep.cu", "quant_v": "prep
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=6000)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=0, help="timed steps (0 = about one second of work)")
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="deit_b")
+    ap.add_argument("--workload", default="sweep32768_d128")
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (small profiling cases)")
     ap.add_argument("--attn-impl", choices=["auto", "simt", "tcgen05"], default="auto")
     ap.add_argument("--rotate", type=int, default=0, help="input sets cycled to defeat L2 (0 = auto)")
@@ -188,6 +190,9 @@ def oracle_sample(w, budget_s: float, threads: int):
     ops = 4.0 * nb * w.H * nr * w.N * w.d
     desc = (f"{nb} of {w.B} batches x {w.H} heads, {nr} of {w.N} query rows against all {w.N} keys, "
             f"{threads} threads")
+    if nb < w.B or nr < w.N:
+        desc += ("; extrapolated: the rate over these rows stands for the whole workload (rows are "
+                 "independent and cost the same)")
     return ops, dt, desc
 
 
@@ -263,10 +268,22 @@ def main():
         j = i % R
         ba.attention_fwd(qs[j], ks[j], vs[j], bias, out=outs[j], workspace=wss[j])
 
+    w0 = torch.cuda.Event(enable_timing=True)
+    w1 = torch.cuda.Event(enable_timing=True)
+    w0.record(stream)
     for i in range(args.warmup):
         step(i)
+    w1.record(stream)
     torch.cuda.synchronize()
     impl_used = {1: "simt", 2: "tcgen05"}.get(ba.last_attention_impl(), "?")
+    if args.steps <= 0:  # about one second of timed work, the same count on every rank
+        per = w0.elapsed_time(w1) / max(1, args.warmup)
+        steps = max(20, min(20000, int(1000.0 / max(per, 1e-3))))
+        if world > 1:
+            t = torch.tensor([steps], dtype=torch.int64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MIN)
+            steps = int(t.item())
+        args.steps = steps
 
     clocks = ClockSampler(dev.index)
     clocks.start()

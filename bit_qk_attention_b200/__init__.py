@@ -20,6 +20,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libbinattn.so")
 
 BA_F16, BA_BF16, BA_F32 = 0, 1, 2
+NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024  # BA_NOALLOC_SCRATCH_BYTES of include/binattn.h
 BIAS_NONE, BIAS_DENSE, BIAS_RELPOS2D = 0, 1, 2
 IMPL_AUTO, IMPL_SIMT, IMPL_TCGEN05 = 0, 1, 2
 

@@ -16,6 +16,9 @@
 //     every region is fully written by the first kernels of a call before any kernel reads it.
 //   * The first call on each device looks up the array's device address (cudaGetSymbolAddress,
 //     with that device current) and caches it; make that first call before any stream capture.
+//     The cache assumes the device's primary context lives as long as the process: after a
+//     cudaDeviceReset the library's device memory is reloaded elsewhere and the cached address
+//     is stale, so a process that resets a device must not call this entry point afterwards.
 //   * Problems whose workspace exceeds kScratchBytes are refused with BA_ERR_WORKSPACE before
 //     anything is launched. Nothing here calls cudaMalloc, cudaFree or another allocating routine.
 #include <cuda_runtime.h>

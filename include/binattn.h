@@ -161,7 +161,8 @@ ba_status ba_attention_fwd(const void* q, const void* k, const void* v, ba_dtype
  *     and must be ordered by the caller. Its contents persist between calls; none of it needs
  *     to start at zero.
  *   - The first call on each device looks up the array's device address (and caches it);
- *     make that first call before any stream capture.
+ *     make that first call before any stream capture. The cache assumes the device's primary
+ *     context lives as long as the process (no cudaDeviceReset between calls).
  *   - Allocates nothing: no cudaMalloc, cudaFree or other allocating routine.
  */
 #define BA_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)

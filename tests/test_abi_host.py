@@ -67,6 +67,14 @@ def test_host_queries(L):
         assert L.ba_status_string(s).startswith(b"BA_")
 
 
+def test_noalloc_limit_matches_header():
+    import bit_qk_attention_b200 as ba
+    text = open(HEADER).read()
+    m = re.search(r"#define BA_NOALLOC_SCRATCH_BYTES \((\d+)u \* (\d+)u \* (\d+)u\)", text)
+    assert m, "BA_NOALLOC_SCRATCH_BYTES not found"
+    assert int(m.group(1)) * int(m.group(2)) * int(m.group(3)) == ba.NOALLOC_SCRATCH_BYTES
+
+
 def test_impl_switch(L):
     assert L.ba_set_attention_impl(3) == 1
     assert L.ba_set_attention_impl(1) == 0 and L.ba_get_attention_impl() == 1

@@ -140,6 +140,73 @@ def test_forward_parity(ba, name, nrows, impl):
     assert_o_close(got, want, f"{name} impl={impl}")
 
 
+PACKED_CONFIGS = [("deit_b", None), ("dit256", None), ("dit1024", 32), ("edge", None)]
+
+
+@pytest.mark.parametrize("name,nrows", PACKED_CONFIGS, ids=[c[0] for c in PACKED_CONFIGS])
+def test_packed_path(ba, name, nrows):
+    """The three-call path of the C ABI: ba_pack_signs (q, k), ba_quant_v (v), then
+    ba_attention_fwd_packed, against the oracle: sign words, mu, V codes and scales and the
+    integer logits bit-exact (logits on the shorter cases), O within the bar. The packed operands
+    are then rewritten by a caller kernel (a device copy into fresh buffers that were filled with
+    garbage) directly before a second packed call on the same stream: the attention kernel, which
+    may be launched before the previous kernel of the stream has finished, must see the new
+    contents."""
+    import torch
+    from bit_qk_attention_b200 import inputs
+    w = (inputs.random_case(2, 3, 263, 72, torch.bfloat16, 2, seed=9, grid=(2, 131), n_prefix=1)
+         if name == "edge" else inputs.by_name(name))
+    ba.set_attention_impl(0)
+    o = oracle.get()
+    q, k, v = _dev(w)
+    bq, mq = ba.pack_signs(q)
+    bk, mk = ba.pack_signs(k)
+    vq, vs = ba.quant_v(v)
+    bias = ba.bias_from_workload(w, q.device)
+    small = w.N <= 300
+    res = ba.attention_fwd_packed(bq, mq, bk, mk, vq, vs, w.d, bias, out_dtype=torch.float32, debug_logits=small)
+    out, lg = res if small else (res, None)
+    torch.cuda.synchronize()
+    ba.check_device_status()
+    qf, kf, vf = oracle_qkv(w)
+    assert np.array_equal(bq.cpu().numpy().view(np.uint32), o.pack_signs(qf))
+    assert np.array_equal(bk.cpu().numpy().view(np.uint32), o.pack_signs(kf))
+    np.testing.assert_allclose(mq.cpu().numpy(), o.mu(qf), rtol=3e-6, atol=0)
+    np.testing.assert_allclose(mk.cpu().numpy(), o.mu(kf), rtol=3e-6, atol=0)
+    want_q, want_s = o.quant_v(vf)
+    assert np.array_equal(vq.cpu().numpy()[..., :w.d], want_q) and np.array_equal(vs.cpu().numpy(), want_s)
+    if small:
+        assert np.array_equal(lg.cpu().numpy(), o.logits(o.pack_signs(qf), o.pack_signs(kf), w.d))
+    rows = None if nrows is None else sample_rows(w.N, nrows, seed=w.N + 1)
+    want = oracle_forward(w, rows=rows)
+    got = out.cpu().numpy()
+    assert_o_close(got if rows is None else got[:, :, rows], want, f"packed {name}")
+
+    # Fresh operand buffers full of garbage, rewritten by a device copy right before the call.
+    ops = [bq, mq, bk, mk, vq, vs]
+    fresh = [torch.empty_like(t) for t in ops]
+    for t in fresh:
+        t.view(torch.uint8).fill_(0xA5)
+    torch.cuda.synchronize()
+    for dst, src in zip(fresh, ops):
+        dst.copy_(src)  # a caller's kernel writing the packed operands on the current stream
+    out2 = ba.attention_fwd_packed(*fresh, w.d, bias, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    ba.check_device_status()
+    assert np.array_equal(out2.cpu().numpy(), got), "packed call after a caller kernel on the same stream"
+
+
+@pytest.mark.parametrize("seed", [11, 21, 31, 41, 51])
+def test_deit_b_seeds(ba, seed):
+    """DeiT-B-shaped draws other than the default seed: the x8 outlier channels give peaky rows
+    with a small softmax sum, where one 8-bit P code that differs from the oracle's moves O the
+    most. Full output, every row."""
+    from bit_qk_attention_b200 import inputs
+    w = inputs.deit_b(seed=seed)
+    out = _forward(ba, w, 2).cpu().numpy()
+    assert_o_close(out, oracle_forward(w), f"deit_b seed {seed}")
+
+
 EDGE = [  # B, H, N, d, dtype, bias kind, extra
     (1, 1, 1, 64, "f16", 0, {}), (1, 2, 2, 1, "bf16", 1, {}), (2, 1, 127, 31, "f16", 1, {}),
     (1, 2, 129, 33, "bf16", 2, {"grid": (3, 43)}), (1, 1, 197, 72, "f16", 2, {"grid": (14, 14), "n_prefix": 1}),

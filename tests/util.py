@@ -9,6 +9,14 @@ import oracle
 O_MAX_ABS = 2e-3
 O_MEAN_ABS = 2e-4
 
+# (case, max-abs, mean-abs, P-code mismatches or None, codes compared) per parity check, printed
+# in the terminal summary of the run (tests/conftest.py).
+PARITY_STATS = []
+
+
+def record_parity(case: str, max_abs: float, mean_abs: float, p_mismatch=None, p_total=None):
+    PARITY_STATS.append((case, max_abs, mean_abs, p_mismatch, p_total))
+
 
 def oracle_bias(w) -> "oracle.Bias":
     if w.bias_kind == 0 or w.bias is None:
@@ -44,5 +52,7 @@ def o_errors(got: np.ndarray, want: np.ndarray):
 def assert_o_close(got: np.ndarray, want: np.ndarray, what: str = ""):
     assert np.all(np.isfinite(got)), f"{what}: non-finite output"
     mx, mean = o_errors(got, want)
+    if what:
+        record_parity(what, mx, mean)
     assert mx <= O_MAX_ABS and mean <= O_MEAN_ABS, f"{what}: max-abs {mx:.3g}, mean-abs {mean:.3g}"
     return mx, mean
