@@ -60,6 +60,8 @@ SIGNATURES = {
                                      _I, _P, _P]),
     "ba_attention_fwd": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, ctypes.POINTER(CBias), _F, _P, _I, _P, _SZ,
                               _P, _P]),
+    "ba_attention_fwd_debug": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, ctypes.POINTER(CBias), _F, _P, _I, _P, _SZ,
+                                    _P, _P, _I, _P]),
     "ba_attention_fwd_noalloc": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, ctypes.POINTER(CBias), _F, _P, _I, _P,
                                       _P]),
     "ba_set_attention_impl": (_I, [_I]),
@@ -273,6 +275,27 @@ def attention_fwd(q, k, v, bias: Optional[Bias] = None, softmax_scale: float = 0
                                   float(softmax_scale), _ptr(out), _dt(out), _ptr(workspace),
                                   workspace.numel(), _ptr(dbg), _stream(stream)), "ba_attention_fwd")
     return (out, dbg) if debug_logits else out
+
+
+def attention_fwd_debug(q, k, v, bias: Optional[Bias] = None, softmax_scale: float = 0.0, out_dtype=None,
+                        check_all_codes: bool = False, stream=None):
+    """The whole forward pass with its debug outputs: (O, int32 logits [B,H,N,N], uint8 P codes
+    [B,H,N,N]). check_all_codes recomputes every near-tie code exactly (see ba_attention_fwd_debug)."""
+    torch = _torch()
+    _qkv_check(q, k, v)
+    B, H, N, d = q.shape
+    out = torch.empty((B, H, N, d), dtype=out_dtype or q.dtype, device=q.device)
+    nws = lib().ba_workspace_bytes(B, H, N, d)
+    nws = 0 if nws == ctypes.c_size_t(-1).value else nws
+    workspace = torch.empty(max(nws, 1), dtype=torch.uint8, device=q.device)
+    dbg = torch.empty((B, H, N, N), dtype=torch.int32, device=q.device)
+    dbg_p = torch.empty((B, H, N, N), dtype=torch.uint8, device=q.device)
+    cb = (bias or Bias()).c()
+    _check(lib().ba_attention_fwd_debug(_ptr(q), _ptr(k), _ptr(v), _dt(q), B, H, N, d, ctypes.byref(cb),
+                                        float(softmax_scale), _ptr(out), _dt(out), _ptr(workspace),
+                                        workspace.numel(), _ptr(dbg), _ptr(dbg_p), 1 if check_all_codes else 0,
+                                        _stream(stream)), "ba_attention_fwd_debug")
+    return out, dbg, dbg_p
 
 
 def bias_from_workload(w, device) -> Optional[Bias]:

@@ -323,10 +323,13 @@ ba_status ba_attention_fwd_packed(const uint32_t* bits_q, const float* mu_q, con
   return run_attention(ap, static_cast<cudaStream_t>(stream));
 }
 
-ba_status ba_attention_fwd(const void* q, const void* k, const void* v, ba_dtype dt, int B, int H,
-                           int N, int d, const ba_bias* bias, float softmax_scale, void* o,
-                           ba_dtype o_dt, void* ws, size_t ws_bytes, int32_t* dbg_logits,
-                           void* stream) {
+}  // extern "C"
+
+namespace {
+
+ba_status forward(const void* q, const void* k, const void* v, ba_dtype dt, int B, int H, int N, int d,
+                  const ba_bias* bias, float softmax_scale, void* o, ba_dtype o_dt, void* ws, size_t ws_bytes,
+                  int32_t* dbg_logits, uint8_t* dbg_p, int p_check_all, void* stream) {
   ba_status st = check_dims(B, H, N, d);
   if (st != BA_OK) return st;
   if (dt != BA_F16 && dt != BA_BF16) return BA_ERR_INVALID_ARG;
@@ -411,10 +414,34 @@ ba_status ba_attention_fwd(const void* q, const void* k, const void* v, ba_dtype
   ap.o = o;
   ap.o_dt = o_dt;
   ap.dbg_logits = dbg_logits;
+  ap.dbg_p = dbg_p;
+  ap.p_check_all = p_check_all;
   st = run_attention(ap, s);
   record(ev, 4, s);
   keep(ev, st == BA_OK);
   return st;
+}
+
+}  // namespace
+
+extern "C" {
+
+ba_status ba_attention_fwd(const void* q, const void* k, const void* v, ba_dtype dt, int B, int H,
+                           int N, int d, const ba_bias* bias, float softmax_scale, void* o,
+                           ba_dtype o_dt, void* ws, size_t ws_bytes, int32_t* dbg_logits,
+                           void* stream) {
+  return forward(q, k, v, dt, B, H, N, d, bias, softmax_scale, o, o_dt, ws, ws_bytes, dbg_logits, nullptr, 0,
+                 stream);
+}
+
+ba_status ba_attention_fwd_debug(const void* q, const void* k, const void* v, ba_dtype dt, int B, int H,
+                                 int N, int d, const ba_bias* bias, float softmax_scale, void* o,
+                                 ba_dtype o_dt, void* ws, size_t ws_bytes, int32_t* dbg_logits,
+                                 uint8_t* dbg_p, int check_all_codes, void* stream) {
+  if (check_all_codes != 0 && check_all_codes != 1) return BA_ERR_INVALID_ARG;
+  if (!aligned16(dbg_p)) return BA_ERR_ALIGNMENT;
+  return forward(q, k, v, dt, B, H, N, d, bias, softmax_scale, o, o_dt, ws, ws_bytes, dbg_logits, dbg_p,
+                 check_all_codes, stream);
 }
 
 ba_status ba_stage_timing(int enable) {

@@ -108,6 +108,7 @@ __global__ void __launch_bounds__(kThreads) attn_simt_kernel(AttnParams p) {
         code = min(255, max(0, __float2int_rn(__fmul_rn(255.0f, pf))));
       }
       sp_b[r * (kRowWords * 4) + j] = static_cast<uint8_t>(code);
+      if (p.dbg_p != nullptr && row_ok && j < nk) p.dbg_p[(bh * N + i) * N + t0 + j] = static_cast<uint8_t>(code);
     }
     if (row_ok) {
       l = l * c + lsum;

@@ -7,38 +7,40 @@
 // on every page).
 //
 // How, on B200:
-//   * A work item is NQ query tiles of 128 rows of one (b, h): one tile in 256 tensor-memory
-//     columns (two CTAs per SM) when the head and the bias table fit, else two tiles in 512.
-//     For heads up to 80 channels the CTAs are persistent (as many as fit at once): each walks
-//     a list of items, grouped by head when the head's rel-pos table is staged, while its
-//     producers and MMA thread run ahead into the next item (the K/V ring continues across
-//     items; consecutive items start on alternate P.V accumulators, so an item's epilogue
-//     overlaps the next item's first MMAs). Wider heads run one item per CTA
-//     (attn_tc_single_kernel), which measured faster there.
-//   * Warps 2 and 3 expand the 1-bit sign rows of Q (once) and of each K block into fp8 +-1
-//     operands in shared memory (channels >= d become 0); warp 0 TMA-loads the int8 V block
-//     (a 4-D tensor map that lands it in the MN-major core-matrix layout the MMA reads) and
-//     writes the block's rel-pos key offsets. A 4-stage ring of K/V blocks decouples them from
-//     the MMAs.
+//   * A work item is one query tile of 128 rows of one (b, h). Tensor memory holds two S
+//     buffers (fp32, 128 columns each: QK of the next block runs while the softmax works on this
+//     one), the s32 P.V accumulator of one block and the fp32 running output (DP columns each).
+//     One CTA per SM, as many CTAs as SMs, each walking a list of items; its producers and MMA
+//     thread run ahead into the next item.
+//   * Warps 2 and 3 expand the 1-bit sign rows of Q (once per item) and of each K block into
+//     fp8 +-1 operands in shared memory (channels >= d become 0); warp 0 TMA-loads the int8 V
+//     block (a 4-D tensor map that lands it in the MN-major core-matrix layout the MMA reads)
+//     and stages the block's bias data. A 4-stage ring of K/V blocks decouples them from the
+//     MMAs.
 //   * Warp 1 issues the MMAs from one thread:
-//       S  = Q . K^T   tcgen05.mma kind::f8f6f4 (e4m3 +-1, fp32 accumulate: exact integers)
-//       O += P . V     tcgen05.mma kind::i8, A = the uint8 codes read from TMEM, B = int8 V
-//     both accumulators live in tensor memory.
-//   * Warpgroup 1+q (one thread per query row) runs the softmax of query tile q: it reads its
-//     row of S from TMEM, forms s = fmaf(alpha, x, b), the running max, P~ = 2^((s-m) log2 e),
-//     the row sum, and writes the 8-bit codes back to TMEM as the A operand of P.V.
-//   * The int32 P.V accumulator keeps accumulating across key blocks while no row of the tile
-//     raises its running max (every rescale factor is exactly 1 then). When a row's max rises,
-//     P.V of that block starts the tile's second accumulator instead, and while the MMAs run
-//     the softmax threads fold the first one into their fp32 running outputs,
-//     O~ = (O~ + acc) * exp(m_old - m_new) (factor 1 for rows whose max did not rise). This is
-//     the same arithmetic as rescaling every block, off the softmax's critical path.
+//       S    = Q . K^T   tcgen05.mma kind::f8f6f4 (e4m3 +-1, fp32 accumulate: exact integers)
+//       acc  = P . V     tcgen05.mma kind::i8, A = the uint8 codes read from TMEM, B = int8 V
+//     both accumulators live in tensor memory; acc holds one block's product.
+//   * Two softmax warpgroups per tile: thread (half h, row r) takes keys 64h .. 64h + 63 of
+//     every block for query row r. It reads its half row of S from TMEM, forms
+//     s = fmaf(alpha, x, b), exchanges its partial maximum with its partner thread (a
+//     two-warp mbarrier), and computes P~ = 2^((s - m) log2 e), its part of the row sum and the
+//     8-bit codes, which it writes back to TMEM as the A operand of P.V.
+//   * Codes that lie within the error band of the fast exponential around a rounding tie are
+//     recomputed from the double-precision exponential, in every block where a changed code
+//     could move the output by a set fraction of the error bar (rows whose running softmax sum
+//     is still small relative to the head's largest V scale), or everywhere on request.
+//   * The running output lives in tensor memory as F' = O~ / g (g the product of the row's
+//     rescale factors since the item began), so folding a block's integer product in is one
+//     FMA per element, F' += acc / g, with the product converted exactly through the bit
+//     pattern of 1.5 * 2^23 (a block's |acc| <= 255 * 127 * 128 < 2^22).
 //   * Every wait is bounded (1 s): on expiry the kernel records BA_ERR_TIMEOUT in a device
 //     status word, every role leaves its loop, and the CTA frees its tensor memory.
 #include <cuda.h>
 #include <math_constants.h>
 
 #include <algorithm>
+#include <type_traits>
 #include <mutex>
 
 #include "common.cuh"
@@ -53,66 +55,86 @@ namespace {
 
 using namespace ptx;
 
-constexpr int BM = 128;        // query rows per tile = MMA M
-constexpr int BN = kKvBlock;   // keys per block = MMA N of QK, K of P.V
+constexpr int BM = 128;       // query rows per tile = MMA M
+constexpr int BN = kKvBlock;  // keys per block = MMA N of QK, K of P.V
 constexpr uint64_t kTimeoutNs = 1000000000ull;
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr uint32_t kMagicBits = 0x4B400000u;  // bit pattern of 1.5 * 2^23
+constexpr float kMagic = 12582912.0f;         // 1.5 * 2^23
+constexpr int kWinFloats = 1024;              // rel-pos window per (tile, stage)
 
-template <int DP, int NQ_>
+// Bias variants of the kernel.
+constexpr int kBiasNone = 0;
+constexpr int kBiasDense = 1;
+constexpr int kRelSmem = 2;    // rel-pos, the head's whole table staged in shared memory
+constexpr int kRelGlobal = 3;  // rel-pos, table read from global memory
+constexpr int kRelWindow = 4;  // rel-pos on a grid of width 32k without class tokens: per (tile,
+                               // block) window of the table staged by the producer
+__host__ __device__ constexpr bool is_relpos_general(int bk) { return bk == kRelSmem || bk == kRelGlobal; }
+
+template <int DP, int BK>
 struct Cfg {
-  static constexpr int DQ = (DP + 31) / 32 * 32;   // QK contraction width: fp8 K-steps of 32
-  static constexpr int NQ = NQ_;                    // query tiles per CTA
-  static constexpr int kThreads = 128 + 128 * NQ;   // 4 service warps + NQ softmax warpgroups
-  // The fp32 running output F of a row lives in shared memory for heads up to 64 wide (tensor
-  // memory then holds S and two accumulators per tile), else in tensor memory.
-  static constexpr bool kFSmem = DP <= 64;
+  // One 128-row query tile per item and CTA, S double-buffered (QK of the next block runs while
+  // the softmax works on this one). Two tiles with one S buffer each also fit tensor memory for
+  // heads up to 64 channels, but their 640 threads leave the softmax too few registers.
+  static constexpr int NQ = 1;                 // query tiles per item
+  static constexpr int SB = NQ == 1 ? 2 : 1;   // S buffers per tile
+  static constexpr int DQ = (DP + 31) / 32 * 32;  // QK contraction width: fp8 K-steps of 32
+  static constexpr int DH = DP / 2;            // accumulator / output columns per softmax half
+  static constexpr int kThreads = 128 + 256 * NQ;
+  static constexpr int kStages = 4;
   static constexpr int kQBytes = BM * DQ;
   static constexpr int kKBytes = BN * DQ;
   static constexpr int kVBytes = BN * DP;
-  static constexpr int kStages = (NQ == 1 && DP <= 64) ? 3 : 4;  // K/V pipeline depth
+  static constexpr int kWinBytes = BK == kRelWindow ? kStages * NQ * kWinFloats * 4 : 0;
+  static constexpr int kWinKBytes = BK == kRelWindow ? kStages * NQ * 4 * 4 : 0;
+  static constexpr int kKoffBytes = is_relpos_general(BK) ? kStages * BN * 4 : 0;
   static constexpr int offQ = 0;
   static constexpr int offK = offQ + NQ * kQBytes;
   static constexpr int offV = offK + kStages * kKBytes;
-  static constexpr int offKoff = offV + kStages * kVBytes;
-  static constexpr int offScale = offKoff + kStages * BN * 4;  // V scales (single-item kernel)
-  static constexpr int offBar = offScale + 128 * 4;
-  static constexpr int kNumBars = 2 * kStages + 3 + 3 * NQ;
-  static constexpr int offMisc = offBar + kNumBars * 8;           // tmem base, abort flag
-  static constexpr int offVotes = offMisc + 16;                    // [2][NQ][4] u32
-  static constexpr int offF = (offVotes + 2 * NQ * 4 * 4 + 15) / 16 * 16;
-  static constexpr int kFBytes = kFSmem ? NQ * BM * DP * 4 : 0;   // [DP/4][NQ*128] float4
-  static constexpr int kBytes = offF + kFBytes;
-  static constexpr int kTabOff = (kBytes + 127) / 128 * 128;
-  // Tensor-memory columns of query tile q: S (fp32, 128 columns; the softmax overwrites it
-  // with s and then its first 32 columns with the u8 codes P — the MMAs of one CTA run in
-  // issue order, so P.V reads P before the next QK rewrites S), two s32 P.V accumulators
-  // O0/O1 (DP each: P.V switches to the other one when a row's max rises, while the softmax
-  // threads fold the first into F) and, for wide heads, F (fp32, DP).
-  __host__ __device__ static constexpr uint32_t tS(int q) { return q * 256; }
-  __host__ __device__ static constexpr uint32_t tP(int q) { return q * 256; }
-  __host__ __device__ static constexpr uint32_t tO(int q, int b) { return q * 256 + 128 + b * DP; }
-  __host__ __device__ static constexpr uint32_t tF(int q) { return q * 256 + 128 + 2 * DP; }
-  static constexpr int kTmemUsed = tO(NQ - 1, 1) + DP + (kFSmem ? 0 : DP);
-  static_assert(kTmemUsed <= 512, "tensor memory budget");
-  static_assert(NQ == 1 || kFSmem, "two tiles per CTA need F in shared memory");
-  // Columns allocated: a CTA whose tiles fit in half of tensor memory takes 256 columns and
-  // shares its SM with a second CTA.
-  static constexpr int kTmemCols = kTmemUsed <= 256 ? 256 : 512;
-  static constexpr int kCtasPerSm = 512 / kTmemCols;
+  static constexpr int offWin = offV + kStages * kVBytes;  // [S][NQ][kWinFloats] f32
+  static constexpr int offWinK = offWin + kWinBytes;       // [S][NQ][4] s32 chunk offsets
+  static constexpr int offKoff = offWinK + kWinKBytes;     // [S][BN] s32 key offsets
+  static constexpr int offX = offKoff + kKoffBytes;        // per row: m_j [2][BM], L' [BM], m_ref [BM]
+  static constexpr int offBar = offX + 4 * BM * 4;
+  static constexpr int kNumBars = 2 * kStages + 3 + 2 + 2 + 2 + 2 + 1 + 4;
+  static constexpr int offMisc = offBar + kNumBars * 8;  // tmem base, abort flag
+  static constexpr int kBytes = offMisc + 16;
+  static constexpr int kTabOff = (kBytes + 127) / 128 * 128;  // staged rel-pos table (kRelSmem)
+  // Tensor-memory columns of tile q: S buffer b (fp32, 128 columns; the softmax overwrites its
+  // first 32 columns with the uint8 codes P — the MMAs of one CTA run in issue order, so P.V
+  // reads P before the next QK into that buffer rewrites it), the s32 P.V accumulator of one
+  // block (DP) and the fp32 running output F' (DP).
+  __host__ __device__ static constexpr uint32_t tS(int q, int b) { return q * 256 + b * 128; }
+  __host__ __device__ static constexpr uint32_t tAcc(int q) { return q * 256 + SB * 128; }
+  __host__ __device__ static constexpr uint32_t tF(int q) { return tAcc(q) + DP; }
+  static_assert(tF(NQ - 1) + DP <= 512, "tensor memory budget");
+  static_assert(DP % 16 == 0 && DP >= 16 && DP <= 128, "head width");
 };
 
-// Barrier slots: kv_full[S], kv_empty[S], q_full, q_empty, drain, s_full[NQ], p_full[NQ],
-// o_done[NQ]. Phases count K/V blocks (kv_*: per stage; s_full, p_full: per block) or work
-// items (q_*, o_done) across all the items a CTA processes.
-template <int S, int NQ> struct Bars {
+// Barrier slots. Phases count K/V blocks (kv_*: per stage; s_full: per use of the S buffer;
+// p_full, pv_done: per block), work items (q_*) or pair exchanges, across all the items a CTA
+// processes.
+template <class C>
+struct Bars {
+  static constexpr int S = C::kStages, NQ = C::NQ, SB = C::SB;
   __host__ __device__ static constexpr int kvfull(int s) { return s; }
   __host__ __device__ static constexpr int kvempty(int s) { return S + s; }
   __host__ __device__ static constexpr int qfull() { return 2 * S; }
   __host__ __device__ static constexpr int qempty() { return 2 * S + 1; }
   __host__ __device__ static constexpr int drain() { return 2 * S + 2; }
-  __host__ __device__ static constexpr int sfull(int q) { return 2 * S + 3 + q; }
-  __host__ __device__ static constexpr int pfull(int q) { return 2 * S + 3 + NQ + q; }
-  __host__ __device__ static constexpr int odone(int q) { return 2 * S + 3 + 2 * NQ + q; }
+  // s_full per S buffer; p_full, pv_done, fold_done per softmax group g (the blocks j with
+  // j % 2 == g, phase j / 2): a parity wait is exact only while the phase before it has
+  // completed, so every waiter walks the phases of a barrier in order; epi_done per item;
+  // mchain per row quarter (the running maximum passed between the groups, one phase per block).
+  __host__ __device__ static constexpr int sfull(int q, int b) { return 2 * S + 3 + q * SB + b; }
+  __host__ __device__ static constexpr int pfull(int g) { return 2 * S + 5 + g; }
+  __host__ __device__ static constexpr int pvdone(int g) { return 2 * S + 7 + g; }
+  __host__ __device__ static constexpr int folddone(int g) { return 2 * S + 9 + g; }
+  __host__ __device__ static constexpr int epidone() { return 2 * S + 11; }
+  __host__ __device__ static constexpr int mchain(int w4) { return 2 * S + 12 + w4; }
+  static_assert(NQ == 1 && SB == 2, "one tile, two S buffers");
+  static_assert(mchain(3) + 1 == C::kNumBars, "barrier count");
 };
 
 // Work items: NQ query tiles of one (b, h). With the head's rel-pos table staged in shared
@@ -120,7 +142,7 @@ template <int S, int NQ> struct Bars {
 // of head h takes items j, j + k, j + 2k, ... of the B * nqb items of that head (nqb = query
 // blocks per (b, h)), so the table is staged once. Otherwise CTA c takes items c, c + G,
 // c + 2G, ... of all B * H * nqb items (G = gridDim.x), item m covering query block m % nqb of
-// slice m / nqb. Recomputed from the launch geometry where needed.
+// slice m / nqb.
 __device__ __forceinline__ int item_count(bool by_head, int B, int H, int nqb) {
   const int total = by_head ? B * nqb : B * H * nqb;
   const int first = by_head ? static_cast<int>(blockIdx.x) / H : static_cast<int>(blockIdx.x);
@@ -145,12 +167,14 @@ __device__ __forceinline__ void item_at(bool by_head, int it, int H, int nqb, in
 // Waits for the phase of `bar` with the given parity. Gives up after kTimeoutNs (recording the
 // timeout in the device status word and raising the CTA's abort flag) or, when `yield` is set,
 // as soon as another role has raised the abort flag.
+// Between checks the thread sleeps in the barrier wait (up to 20 us, woken when the phase
+// completes), so waiting warps take no issue slots from the working ones.
 __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                              bool yield = true) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
     if (yield && *abort_flag) return false;
     if (globaltimer() - t0 > kTimeoutNs) {
       *abort_flag = 1;
@@ -191,228 +215,103 @@ __device__ __forceinline__ void expand_row(uint8_t* dst, const uint4& b, bool ok
   }
 }
 
-// Bias variants of the kernel: BA_BIAS_NONE, BA_BIAS_DENSE, BA_BIAS_RELPOS2D with the head's
-// table staged in shared memory, and kRelposGlobal with the table read from global memory.
-constexpr int kRelposGlobal = 3;
-__host__ __device__ constexpr bool is_relpos(int bk) { return bk == BA_BIAS_RELPOS2D || bk == kRelposGlobal; }
-
-// Fast path of pass 1 for one 32-key block of one row: bias (dense row, or rel-pos table in
-// shared or global memory), s = alpha * x + b in place, running maxima. PARTIAL masks keys
-// at or past nk to -inf.
-template <int BK, bool PARTIAL>
-__device__ __forceinline__ void fast_block(uint32_t (&x)[32], int c, int nk, float2 alpha2, const float* brow_t,
-                                           uint32_t ko_s, uint32_t tb, const float* grow, int tab_mode,
-                                           float (&mx)[4]) {
-#pragma unroll
-  for (int g = 0; g < 4; ++g) {
-    float bv[8];
-    if (BK == BA_BIAS_DENSE) {
-      const float4* src = reinterpret_cast<const float4*>(brow_t + 32 * c + 8 * g);
-      const float4 v0 = __ldg(src), v1 = __ldg(src + 1);
-      bv[0] = v0.x; bv[1] = v0.y; bv[2] = v0.z; bv[3] = v0.w;
-      bv[4] = v1.x; bv[5] = v1.y; bv[6] = v1.z; bv[7] = v1.w;
-    } else if (is_relpos(BK)) {
-      const int4 o0 = lds_s32x4(ko_s + 4u * (32 * c + 8 * g));
-      const int4 o1 = lds_s32x4(ko_s + 4u * (32 * c + 8 * g + 4));
-      if (BK == BA_BIAS_RELPOS2D) {
-        bv[0] = lds_f32(tb - o0.x); bv[1] = lds_f32(tb - o0.y);
-        bv[2] = lds_f32(tb - o0.z); bv[3] = lds_f32(tb - o0.w);
-        bv[4] = lds_f32(tb - o1.x); bv[5] = lds_f32(tb - o1.y);
-        bv[6] = lds_f32(tb - o1.z); bv[7] = lds_f32(tb - o1.w);
-      } else {
-        bv[0] = __ldg(grow - (o0.x >> 2)); bv[1] = __ldg(grow - (o0.y >> 2));
-        bv[2] = __ldg(grow - (o0.z >> 2)); bv[3] = __ldg(grow - (o0.w >> 2));
-        bv[4] = __ldg(grow - (o1.x >> 2)); bv[5] = __ldg(grow - (o1.y >> 2));
-        bv[6] = __ldg(grow - (o1.z >> 2)); bv[7] = __ldg(grow - (o1.w >> 2));
-      }
-    } else {
-#pragma unroll
-      for (int u = 0; u < 8; ++u) bv[u] = 0.0f;
-    }
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int u = 8 * g + 2 * k;
-      const float2 s2 = __ffma2_rn(alpha2, make_float2(__uint_as_float(x[u]), __uint_as_float(x[u + 1])),
-                                   make_float2(bv[2 * k], bv[2 * k + 1]));
-      float sx = s2.x, sy = s2.y;
-      if (PARTIAL) {
-        if (32 * c + u >= nk) sx = -CUDART_INF_F;
-        if (32 * c + u + 1 >= nk) sy = -CUDART_INF_F;
-      }
-      x[u] = __float_as_uint(sx);
-      x[u + 1] = __float_as_uint(sy);
-      mx[k] = fmax3(mx[k], sx, sy);
-    }
+// Tensor-memory loads and stores of N consecutive columns (N a multiple of 8) of this warp's
+// 32 lanes, split into x32 / x16 / x8 pieces; r points at a register array indexed by
+// constants only.
+template <int N, int O = 0>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t* r) {
+  if constexpr (N - O >= 32) {
+    tmem_ld32p(taddr + O, r + O);
+    tmem_ld_cols<N, O + 32>(taddr, r);
+  } else if constexpr (N - O >= 16) {
+    tmem_ld16p(taddr + O, r + O);
+    tmem_ld_cols<N, O + 16>(taddr, r);
+  } else if constexpr (N - O >= 8) {
+    tmem_ld8p(taddr + O, r + O);
+    tmem_ld_cols<N, O + 8>(taddr, r);
   }
 }
 
-// 2^t for a pair of t <= 0 on the FMA and integer pipes, for the share of the softmax's
-// exponentials that the transcendental unit (which computes the rest, and is the softmax's
-// bottleneck) does not take. t is clamped to -125 (2^-125: a u8 code of 0, a negligible
-// addition to the row sum; masked keys arrive as -inf); j = rint(t) by adding and subtracting
-// 1.5 * 2^23, f = t - j in [-1/2, 1/2]; 2^f by a degree-5 polynomial with c0 = 1 (a weighted
-// least-squares fit in relative error on Chebyshev nodes, bit_qk_attention_b200/exp2_poly.py;
-// at most 1.6e-7 relative error in float32); 2^j is added to the exponent bits: the bit
-// pattern of t + 1.5 * 2^23 holds j in its low bits, and shifted left by 23 it is j << 23.
-__device__ __forceinline__ float2 exp2_poly2(float2 t) {
-  t.x = fmaxf(t.x, -125.0f);
-  t.y = fmaxf(t.y, -125.0f);
-  const float2 r = __fadd2_rn(t, make_float2(12582912.0f, 12582912.0f));
-  const float2 j = __fadd2_rn(r, make_float2(-12582912.0f, -12582912.0f));
-  const float2 f = __ffma2_rn(j, make_float2(-1.0f, -1.0f), t);
-  float2 q = __ffma2_rn(make_float2(1.321867225e-03f, 1.321867225e-03f), f,
-                        make_float2(9.671698324e-03f, 9.671698324e-03f));
-  q = __ffma2_rn(q, f, make_float2(5.550893024e-02f, 5.550893024e-02f));
-  q = __ffma2_rn(q, f, make_float2(2.402223796e-01f, 2.402223796e-01f));
-  q = __ffma2_rn(q, f, make_float2(6.931468844e-01f, 6.931468844e-01f));
-  q = __ffma2_rn(q, f, make_float2(1.0f, 1.0f));
-  return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(r.x) << 23)),
-                     __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(r.y) << 23)));
-}
-
-// Pairs (of the 16 in a 32-key chunk) whose exponentials take the polynomial: the bits of
-// kPolyPairs, spread over the chunk. Off by default: a quarter measured 2-4 % faster on B200,
-// but any fast exponential can move a u8 code across a rounding tie relative to the exact
-// exp(s - m), and which codes move depends on the mix; the default keeps one implementation
-// (the hardware ex2) for every logit.
-#ifndef BA_POLY_PAIRS
-#define BA_POLY_PAIRS 0x0u
-#endif
-constexpr uint32_t kPolyPairs = BA_POLY_PAIRS;
-
-// Folding an s32 P.V accumulator row into the fp32 running output of the row:
-// F = (F + acc) * ct, in groups of NC chunks of 16 columns starting at chunk C0. fold_load
-// issues a group's tensor-memory loads (the accumulator, and F when it lives in tensor
-// memory); fold_finish waits for them and completes the group. `fresh`: F holds nothing yet
-// (read as 0). `one_block`: the accumulator holds a single block's P.V,
-// |acc| <= 255 * 127 * 128 < 2^22, which converts exactly by adding it to the bit pattern of
-// 1.5 * 2^23 and subtracting that value as a float; otherwise the hardware conversion is used.
-// F lives in shared memory ([DP/4][NQ*128] float4, `fr` = this row's first entry) or in tensor
-// memory (`aF`).
-template <class C>
-struct FoldShape {
-  static constexpr int NCH = C::kVBytes / BN / 16;  // chunks per row
-  // 2 chunks (32 columns) per group when F is in shared memory (those CTAs share an SM: 128
-  // 2 chunks (32 columns) per group when F is in shared memory (those CTAs share an SM: 128
-  // registers per thread), 4 when it is in tensor memory (one CTA per SM).
-  static constexpr int G = C::kFSmem ? 2 : 4;
-  __host__ __device__ static constexpr int nc(int c0) { return (NCH - c0 < G) ? NCH - c0 : G; }
-};
-
-template <class C, int C0, int NC>
-__device__ __forceinline__ void fold_load(uint32_t acc, uint32_t aF, bool fresh, uint32_t (&a)[NC][16],
-                                          uint32_t (&fb)[NC][16]) {
-#pragma unroll
-  for (int k = 0; k < NC; ++k) {
-    tmem_ld16(acc + 16 * (C0 + k), a[k]);
-    if (!C::kFSmem && !fresh) tmem_ld16(aF + 16 * (C0 + k), fb[k]);
+template <int N, int O = 0>
+__device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const uint32_t* r) {
+  if constexpr (N - O >= 32) {
+    tmem_st32p(taddr + O, r + O);
+    tmem_st_cols<N, O + 32>(taddr, r);
+  } else if constexpr (N - O >= 16) {
+    tmem_st16p(taddr + O, r + O);
+    tmem_st_cols<N, O + 16>(taddr, r);
+  } else if constexpr (N - O >= 8) {
+    tmem_st8p(taddr + O, r + O);
+    tmem_st_cols<N, O + 8>(taddr, r);
   }
 }
 
-template <class C, int C0, int NC>
-__device__ __forceinline__ void fold_finish(uint32_t aF, float4* fr, float2 ct2, bool fresh, bool one_block,
-                                            uint32_t (&a)[NC][16], uint32_t (&fb)[NC][16]) {
-  tmem_ld_wait();
-#pragma unroll
-  for (int k = 0; k < NC; ++k) {
-    reg_fence16(a[k]);
-    if (!C::kFSmem && !fresh) reg_fence16(fb[k]);
-  }
-#pragma unroll
-  for (int k = 0; k < NC; ++k) {
-    float f[16];
-    if constexpr (C::kFSmem) {
-#pragma unroll
-      for (int k4 = 0; k4 < 4; ++k4) {
-        const float4 v = fresh ? make_float4(0.0f, 0.0f, 0.0f, 0.0f) : fr[(4 * (C0 + k) + k4) * (C::NQ * BM)];
-        f[4 * k4] = v.x; f[4 * k4 + 1] = v.y; f[4 * k4 + 2] = v.z; f[4 * k4 + 3] = v.w;
-      }
-    } else {
-#pragma unroll
-      for (int e = 0; e < 16; ++e) f[e] = fresh ? 0.0f : __uint_as_float(fb[k][e]);
-    }
-#pragma unroll
-    for (int e = 0; e < 16; e += 2) {
-      float2 av;
-      if (one_block) {
-        av = __fadd2_rn(make_float2(__uint_as_float(a[k][e] + 0x4B400000u), __uint_as_float(a[k][e + 1] + 0x4B400000u)),
-                        make_float2(-12582912.0f, -12582912.0f));
-      } else {
-        av = make_float2(__int2float_rn(static_cast<int>(a[k][e])), __int2float_rn(static_cast<int>(a[k][e + 1])));
-      }
-      const float2 v = __fmul2_rn(__fadd2_rn(make_float2(f[e], f[e + 1]), av), ct2);
-      f[e] = v.x; f[e + 1] = v.y;
-    }
-    if constexpr (C::kFSmem) {
-#pragma unroll
-      for (int k4 = 0; k4 < 4; ++k4)
-        fr[(4 * (C0 + k) + k4) * (C::NQ * BM)] = make_float4(f[4 * k4], f[4 * k4 + 1], f[4 * k4 + 2], f[4 * k4 + 3]);
-    } else {
-#pragma unroll
-      for (int e = 0; e < 16; ++e) fb[k][e] = __float_as_uint(f[e]);
-      tmem_st16(aF + 16 * (C0 + k), fb[k]);
-    }
+// Re-defines registers after tmem_ld_wait() so that no use of a loaded value is scheduled
+// before the wait.
+template <int N, int O = 0>
+__device__ __forceinline__ void reg_fence_cols(uint32_t* r) {
+  if constexpr (O < N) {
+    reg_fence8(r + O);
+    reg_fence_cols<N, O + 8>(r);
   }
 }
 
-// The groups from chunk C0 to the end of the row.
-template <class C, int C0>
-__device__ __forceinline__ void fold_rest(uint32_t acc, uint32_t aF, float4* fr, float2 ct2, bool fresh,
-                                          bool one_block) {
-  if constexpr (C0 < FoldShape<C>::NCH) {
-    constexpr int NC = FoldShape<C>::nc(C0);
-    uint32_t a[NC][16], fb[NC][16];
-    fold_load<C, C0, NC>(acc, aF, fresh, a, fb);
-    fold_finish<C, C0, NC>(aF, fr, ct2, fresh, one_block, a, fb);
-    fold_rest<C, C0 + NC>(acc, aF, fr, ct2, fresh, one_block);
-  }
+// The 8-bit code of one logit taken exactly as the definition states: P~ = exp(s - m) in double
+// rounded to fp32, 255 P~ rounded to fp32, then to the nearest integer (ties to even).
+__device__ __forceinline__ uint32_t exact_code(float s, float m) {
+  const float pe = static_cast<float>(exp(static_cast<double>(s) - static_cast<double>(m)));
+  const int c = __float2int_rn(__fmul_rn(255.0f, pe));
+  return static_cast<uint32_t>(min(255, max(0, c)));
 }
 
-template <int DP, int BK, int NQ_>
-__global__ void __launch_bounds__(Cfg<DP, NQ_>::kThreads, Cfg<DP, NQ_>::kCtasPerSm)
+template <int DP, int BK>
+__global__ void __launch_bounds__(Cfg<DP, BK>::kThreads, 1)
     attn_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmap_v, int tab_mode, int tsize,
-                   int kmax) {
-  using C = Cfg<DP, NQ_>;
-  constexpr int NQ = C::NQ, DQ = C::DQ, S = C::kStages;
-  using Bar = Bars<S, NQ>;
+                   int kmax, int win_stride) {
+  using C = Cfg<DP, BK>;
+  constexpr int NQ = C::NQ, SB = C::SB, DQ = C::DQ, DH = C::DH, S = C::kStages;
+  using Bar = Bars<C>;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // 1024-byte aligned base, derived from the __shared__ array by an offset (not through an integer
+  // cast), so that the compiler keeps every access through it a shared-memory access.
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* sQ = smem + C::offQ;
   uint8_t* sK = smem + C::offK;
   uint8_t* sV = smem + C::offV;
+  float* swin = reinterpret_cast<float*>(smem + C::offWin);
+  int* swink = reinterpret_cast<int*>(smem + C::offWinK);
   int* koff = reinterpret_cast<int*>(smem + C::offKoff);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::offBar);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::offMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::offMisc + 4);
-  // Per block parity, tile and softmax warp: whether a row of that warp raised its max.
-  uint32_t* votes = reinterpret_cast<uint32_t*>(smem + C::offVotes);
-  float4* sF = reinterpret_cast<float4*>(smem + C::offF);  // [DP/4][NQ*128]
-  // Rel-pos table of this CTA's head, staged when it fits: tab_mode 1 = table only,
-  // 2 = table followed by 2*tsize zeros (targets of prefix rows and prefix keys).
+  // Rel-pos table of this CTA's head (kRelSmem): tab_mode 1 = table only, 2 = table followed by
+  // 2*tsize zeros (targets of class-token rows and keys).
   float* stab = reinterpret_cast<float*>(smem + C::kTabOff);
 
   const int N = p.N, d = p.d;
   const int nqb = static_cast<int>(ceil_div(N, BM * NQ));
-  // Items grouped by head when the head's rel-pos table is staged in shared memory.
-  const bool by_head = is_relpos(BK) && tab_mode != 0;
+  const bool by_head = BK == kRelSmem;
   const int n_items = item_count(by_head, p.B, p.H, nqb);
   const int T = static_cast<int>(ceil_div(N, BN));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int st = 0; st < C::kStages; ++st) {
-      // kv_full: the V copy's expect_tx arrival + warp 0 (key offsets) + the two expanding warps.
+    for (int st = 0; st < S; ++st) {
+      // kv_full: the V copy's expect_tx arrival + warp 0 (bias data) + the two expanding warps.
       mbar_init(&bars[Bar::kvfull(st)], 4);
       mbar_init(&bars[Bar::kvempty(st)], 1);
     }
     mbar_init(&bars[Bar::qfull()], 2);
     mbar_init(&bars[Bar::qempty()], 1);
     mbar_init(&bars[Bar::drain()], 1);
-    for (int q = 0; q < NQ; ++q) {
-      mbar_init(&bars[Bar::sfull(q)], 1);
-      mbar_init(&bars[Bar::pfull(q)], 4);
-      mbar_init(&bars[Bar::odone(q)], 1);
+    for (int b = 0; b < SB; ++b) mbar_init(&bars[Bar::sfull(0, b)], 1);
+    for (int g = 0; g < 2; ++g) mbar_init(&bars[Bar::pfull(g)], 4);  // the group's four warps
+    for (int g = 0; g < 2; ++g) {
+      mbar_init(&bars[Bar::pvdone(g)], 1);
+      mbar_init(&bars[Bar::folddone(g)], 4);  // the folding group's four warps
     }
+    mbar_init(&bars[Bar::epidone()], 8);   // both groups
+    for (int w4 = 0; w4 < 4; ++w4) mbar_init(&bars[Bar::mchain(w4)], 1);
     *abort_flag = 0;
     mbar_fence_init();
     fence_proxy_async_smem();
@@ -422,54 +321,33 @@ __global__ void __launch_bounds__(Cfg<DP, NQ_>::kThreads, Cfg<DP, NQ_>::kCtasPer
   // rows, mu and int8 V, which the preparation kernel before it in the stream may still be
   // writing when this kernel was launched as its programmatic dependent.
   grid_dependency_wait();
-  // Warps 2 and 3 load the sign rows of their Q rows and of key block 0 of the first item
-  // before the setup barrier, so the loads overlap the setup.
-  const uint4 zero4 = make_uint4(0u, 0u, 0u, 0u);
-  uint4 pre_q[NQ][2], pre_k[2];
-  if ((warp == 2 || warp == 3) && n_items > 0) {
-    const int half = warp - 2;
-    int64_t bh;
-    int q0;
-    item_at(by_head, 0, p.H, nqb, BM * NQ, bh, q0);
-    const uint4* qrows = reinterpret_cast<const uint4*>(p.bits_q) + bh * N;
-    const uint4* krows = reinterpret_cast<const uint4*>(p.bits_k) + bh * N;
-#pragma unroll
-    for (int q = 0; q < NQ; ++q)
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int row = q0 + q * BM + 64 * half + lane + 32 * u;
-        pre_q[q][u] = row < N ? __ldg(qrows + row) : zero4;
-      }
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int row = 64 * half + lane + 32 * u;
-      pre_k[u] = row < N ? __ldg(krows + row) : zero4;
-    }
-  }
   if (by_head) {
     const float* src = p.bias.data + static_cast<int64_t>(blockIdx.x % p.H) * tsize;
     const int n = (tab_mode == 2) ? 3 * tsize : tsize;
     for (int e = threadIdx.x; e < n; e += C::kThreads) stab[e] = (e < tsize) ? __ldg(src + e) : 0.0f;
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  const uint4 zero4 = make_uint4(0u, 0u, 0u, 0u);
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer: V blocks, key offsets
+    // ------------------------------------------------------------ producer: V blocks, bias data
     // Blocks are counted across the items (g): stage g % S, phase g / S.
     const int W2 = 2 * p.bias.table_w - 1;
+    const int gw = p.bias.grid_w;
     int g = 0;
     bool ok = true;
     for (int it = 0; it < n_items && ok; ++it) {
       int64_t bh;
       int q0;
       item_at(by_head, it, p.H, nqb, BM * NQ, bh, q0);
+      const int h = static_cast<int>(bh % p.H);
       for (int t = 0; t < T; ++t, ++g) {
         const int st = g % S;
         if (g >= S && !wait_warp(&bars[Bar::kvempty(st)], ((g / S) - 1) & 1, abort_flag)) {
@@ -480,25 +358,78 @@ __global__ void __launch_bounds__(Cfg<DP, NQ_>::kThreads, Cfg<DP, NQ_>::kCtasPer
           mbar_arrive_expect_tx(&bars[Bar::kvfull(st)], C::kVBytes);
           tma_load_4d(sV + st * C::kVBytes, &tmap_v, &bars[Bar::kvfull(st)], 0, t * BN, 0, static_cast<int>(bh));
         }
-        if (is_relpos(BK)) {
+        if constexpr (is_relpos_general(BK)) {
 #pragma unroll
           for (int u = 0; u < BN / 32; ++u) {
             const int j = lane + 32 * u, tok = t * BN + j;
             // Keys past N read a valid entry (their P is masked); prefix keys read the zeros
-            // after the staged table (or are marked -1 for the general path).
+            // after the staged table (or are marked -1 for the per-key test).
             int v = (tab_mode == 2) ? -tsize : -1;
             if (tok >= N) {
               v = 0;
             } else if (tok >= p.bias.n_prefix) {
               const int tj = tok - p.bias.n_prefix;
-              const int yj = tj / p.bias.grid_w;
-              v = yj * W2 + (tj - yj * p.bias.grid_w);
+              const int yj = tj / gw;
+              v = yj * W2 + (tj - yj * gw);
             }
-            koff[st * BN + j] = 4 * v;  // byte offset into the staged table
+            koff[st * BN + j] = v;
+          }
+        } else if constexpr (BK == kRelWindow) {
+          // For each tile: the rectangle of (dy, dx) offsets that its rows and this block's keys
+          // form, copied from the head's table with row stride win_stride, and for each 32-key
+          // chunk (one grid row) the offset K_c with which a query row reads its bias as
+          // window[A_i - K_c - u], A_i = y_i * win_stride + x_i.
+          const float* tab = p.bias.data + static_cast<int64_t>(h) * tsize;
+          const int j0 = t * BN, j1 = min(j0 + BN, N) - 1;
+          const int yk_lo = j0 / gw, yk_hi = j1 / gw;
+          const int xk_min = yk_hi > yk_lo ? 0 : j0 - yk_lo * gw;
+          const int xk_max = yk_hi > yk_lo ? gw - 1 : j1 - yk_lo * gw;
+#pragma unroll 1
+          for (int qq = 0; qq < NQ; ++qq) {
+            const int i0 = min(q0 + qq * BM, N - 1), i1 = min(q0 + qq * BM + BM - 1, N - 1);
+            const int yq_lo = i0 / gw, yq_hi = i1 / gw;
+            const int xq_min = yq_hi > yq_lo ? 0 : i0 - yq_lo * gw;
+            const int xq_max = yq_hi > yq_lo ? gw - 1 : i1 - yq_lo * gw;
+            const int dy_lo = yq_lo - yk_hi, ndy = (yq_hi - yq_lo) + (yk_hi - yk_lo) + 1;
+            const int dx_lo = xq_min - xk_max, width = (xq_max - xq_min) + (xk_max - xk_min) + 1;
+            float* win = swin + (st * NQ + qq) * kWinFloats;
+            // The ndy x width entries in batches of 8 loads per lane, all in flight before any is
+            // stored (width >= 32, so a lane's next entry is at most one window row further).
+            const float* tab0 = tab + static_cast<int64_t>(dy_lo + p.bias.table_h - 1) * W2 + (dx_lo + p.bias.table_w - 1);
+            int rr = 0, cc = lane;
+            while (rr < ndy) {
+              float v[8];
+              int dst[8];
+#pragma unroll
+              for (int k = 0; k < 8; ++k) {
+                dst[k] = rr < ndy ? rr * win_stride + cc : -1;
+                if (rr < ndy) v[k] = __ldg(tab0 + static_cast<int64_t>(rr) * W2 + cc);
+                cc += 32;
+                if (cc >= width) {
+                  cc -= width;
+                  ++rr;
+                }
+              }
+#pragma unroll
+              for (int k = 0; k < 8; ++k)
+                if (dst[k] >= 0) win[dst[k]] = v[k];
+            }
+            if (lane < BN / 32) {
+              const int jc = j0 + 32 * lane;
+              const int yk = jc / gw;
+              swink[(st * NQ + qq) * 4 + lane] =
+                  jc < N ? (yk + dy_lo) * win_stride + (jc - yk * gw) + dx_lo : 0;
+            }
           }
         }
         __syncwarp();
+#ifdef BA_TEST_SKIP_ARRIVE
+        // Test build only: the first block's arrival is withheld, so every wait on it runs into
+        // its time limit and the kernel reports BA_ERR_TIMEOUT.
+        if (lane == 0 && g != 0) mbar_arrive(&bars[Bar::kvfull(st)]);
+#else
         if (lane == 0) mbar_arrive(&bars[Bar::kvfull(st)]);
+#endif
       }
     }
     // Leave no TMA copy in flight: wait (bounded, even after an abort) for the stages this
@@ -512,21 +443,29 @@ __global__ void __launch_bounds__(Cfg<DP, NQ_>::kThreads, Cfg<DP, NQ_>::kCtasPer
     const int half = warp - 2;
     int g = 0;
     bool ok = true;
-    uint4 nb[2] = {pre_k[0], pre_k[1]};
+    uint4 nb[2] = {zero4, zero4};
+    uint4 pre_q[NQ][2];
     for (int it = 0; it < n_items && ok; ++it) {
       int64_t bh;
       int q0;
       item_at(by_head, it, p.H, nqb, BM * NQ, bh, q0);
-      if (it > 0) {
-        const uint4* qrows = reinterpret_cast<const uint4*>(p.bits_q) + bh * N;
+      const uint4* qrows = reinterpret_cast<const uint4*>(p.bits_q) + bh * N;
 #pragma unroll
-        for (int q = 0; q < NQ; ++q)
+      for (int q = 0; q < NQ; ++q)
 #pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int row = q0 + q * BM + 64 * half + lane + 32 * u;
-            pre_q[q][u] = row < N ? __ldg(qrows + row) : zero4;
-          }
-        if (!wait_warp(&bars[Bar::qempty()], (it - 1) & 1, abort_flag)) break;
+        for (int u = 0; u < 2; ++u) {
+          const int row = q0 + q * BM + 64 * half + lane + 32 * u;
+          pre_q[q][u] = row < N ? __ldg(qrows + row) : zero4;
+        }
+      if (it == 0) {
+        const uint4* krows = reinterpret_cast<const uint4*>(p.bits_k) + bh * N;
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int row = 64 * half + lane + 32 * u;
+          nb[u] = row < N ? __ldg(krows + row) : zero4;
+        }
+      } else if (!wait_warp(&bars[Bar::qempty()], (it - 1) & 1, abort_flag)) {
+        break;
       }
 #pragma unroll
       for (int q = 0; q < NQ; ++q)
@@ -577,858 +516,517 @@ __global__ void __launch_bounds__(Cfg<DP, NQ_>::kThreads, Cfg<DP, NQ_>::kCtasPer
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    // Per block n (counted across items): P.V of block n-1 first (it needs no new operands),
-    // then QK of block n into the same S columns (issue order keeps P read before S is
-    // rewritten). The first P.V of an item starts the tile's other accumulator, so the previous
-    // item's epilogue can still read the one it ended in.
+    // In order over the blocks j (counted across items): P.V(j) once group j % 2 has written
+    // P(j) and the fold of block j - 1 has read the accumulator; then QK(j + 2) into the S buffer
+    // that P(j) occupied (issue order keeps P read before S is rewritten). QK(0) and QK(1) first.
     if (lane == 0) {
       const uint32_t idesc_qk = (1u << 4) | (0u << 7) | (0u << 10) | (static_cast<uint32_t>(BN >> 3) << 17) |
                                 (static_cast<uint32_t>(BM >> 4) << 24);
       const uint32_t idesc_pv = (2u << 4) | (0u << 7) | (1u << 10) | (1u << 16) |
                                 (static_cast<uint32_t>(DP >> 3) << 17) | (static_cast<uint32_t>(BM >> 4) << 24);
-      bool ok = true;
-      uint32_t cur_acc = (1u << NQ) - 1u;  // bit q: the accumulator P.V of tile q adds into
       const int nblocks = n_items * T;
-      // Step n: P.V of block n - 1 (if n > 0), then QK of block n (if n < nblocks); t is the
-      // item-relative index of block n.
-      for (int n = 0, it = 0, t = 0; n <= nblocks && ok; ++n) {
-        if (n < nblocks && t == 0) {
-          if (!wait_bounded(&bars[Bar::qfull()], it & 1, abort_flag)) {
-            ok = false;
-            break;
-          }
+      auto qk = [&](int j) -> bool {
+        const int t = j % T;
+        if (t == 0) {
+          if (!wait_bounded(&bars[Bar::qfull()], (j / T) & 1, abort_flag)) return false;
           tc_fence_after();
         }
-        const int tp = (t == 0 ? T : t) - 1;  // item-relative index of block n - 1
-        for (int q = 0; q < NQ && ok; ++q) {
-          if (n > 0) {
-            if (!wait_bounded(&bars[Bar::pfull(q)], (n - 1) & 1, abort_flag)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            // Switch to the other accumulator (overwriting it) at an item's first block and
-            // when a row of the tile raised its max: the softmax warps' votes, written before
-            // their p_full arrivals.
-            bool fresh = tp == 0;
-            if (!fresh) {
-              const volatile uint32_t* vt = votes + (((n - 1) & 1) * NQ + q) * 4;
-              fresh = (vt[0] | vt[1] | vt[2] | vt[3]) != 0u;
-            }
-            if (fresh) cur_acc ^= 1u << q;
-            const uint32_t acc = tmem + C::tO(q, (cur_acc >> q) & 1u);
-            const uint32_t vbase = smem_u32(sV + ((n - 1) % S) * C::kVBytes);
+        if (!wait_bounded(&bars[Bar::kvfull(j % S)], (j / S) & 1, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t qb = smem_u32(sQ), kb = smem_u32(sK + (j % S) * C::kKBytes);
 #pragma unroll
-            for (int kk = 0; kk < BN / 32; ++kk)
-              mma_i8_ts(acc, tmem + C::tP(q) + 8 * kk, smem_desc(vbase + 512 * kk, 128, 2048), idesc_pv,
-                        (fresh && kk == 0) ? 0u : 1u);
-            if (tp == T - 1) tc_commit(&bars[Bar::odone(q)]);
-          }
-          if (n < nblocks) {
-            if (q == 0) {
-              if (!wait_bounded(&bars[Bar::kvfull(n % S)], (n / S) & 1, abort_flag)) {
-                ok = false;
-                break;
-              }
-              tc_fence_after();
-            }
-            const uint32_t qb = smem_u32(sQ + q * C::kQBytes), kb = smem_u32(sK + (n % S) * C::kKBytes);
+        for (int kk = 0; kk < DQ / 32; ++kk)
+          mma_f8f6f4_ss(tmem + C::tS(0, j & 1), smem_desc(qb + kk * 4096, 2048, 128),
+                        smem_desc(kb + kk * 4096, 2048, 128), idesc_qk, kk > 0 ? 1u : 0u);
+        tc_commit(&bars[Bar::sfull(0, j & 1)]);
+        if (t == T - 1) tc_commit(&bars[Bar::qempty()]);  // the item's Q tile is free
+        return true;
+      };
+      bool ok = nblocks == 0 || qk(0);
+      if (ok && nblocks > 1) ok = qk(1);
+      for (int j = 0; j < nblocks && ok; ++j) {
+        if (!wait_bounded(&bars[Bar::pfull(j & 1)], (j >> 1) & 1, abort_flag)) break;
+        if (j > 0 && !wait_bounded(&bars[Bar::folddone((j - 1) & 1)], ((j - 1) >> 1) & 1, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t vbase = smem_u32(sV + (j % S) * C::kVBytes);
 #pragma unroll
-            for (int kk = 0; kk < DQ / 32; ++kk)
-              mma_f8f6f4_ss(tmem + C::tS(q), smem_desc(qb + kk * 4096, 2048, 128),
-                            smem_desc(kb + kk * 4096, 2048, 128), idesc_qk, kk > 0 ? 1u : 0u);
-            tc_commit(&bars[Bar::sfull(q)]);
-          }
-        }
-        if (!ok) break;
-        if (n > 0) tc_commit(&bars[Bar::kvempty((n - 1) % S)]);
-        // The item's Q tiles are free once its last QKs have read them.
-        if (n < nblocks && t == T - 1) tc_commit(&bars[Bar::qempty()]);
-        if (++t == T) {
-          t = 0;
-          ++it;
-        }
+        for (int kk = 0; kk < BN / 32; ++kk)
+          mma_i8_ts(tmem + C::tAcc(0), tmem + C::tS(0, j & 1) + 8 * kk, smem_desc(vbase + 512 * kk, 128, 2048),
+                    idesc_pv, kk > 0 ? 1u : 0u);
+        tc_commit(&bars[Bar::pvdone(j & 1)]);
+        tc_commit(&bars[Bar::kvempty(j % S)]);
+        if (j + 2 < nblocks && !qk(j + 2)) break;
       }
       // Every MMA this thread issued has completed before tensor memory is released.
       tc_commit(&bars[Bar::drain()]);
       wait_bounded(&bars[Bar::drain()], 0, abort_flag, false);
     }
     __syncwarp();
-  } else if (warp >= 4) {
+  } else {
     // ------------------------------------------------------------ softmax warpgroups
-    const int q = (warp - 4) >> 2, w4 = warp & 3;
+    // Group g (warps 4 + 4g .. 7 + 4g) takes the key blocks j with j % 2 == g, one thread per
+    // query row (warp w reads tensor-memory lanes 32 (w % 4) ..). While one group evaluates the
+    // exponentials of its block, the other forms the logits of the next: the two phases use
+    // different units (transcendental unit against shared-memory loads) and overlap.
+    //   * The running maximum passes from group to group: the group of block j waits for m_{j-1}
+    //     (mchain), forms m_j and publishes it.
+    //   * Each block is weighted by e_j = exp(m_j - m_ref) against a per-row reference m_ref
+    //     (the item's first block maximum, moved up when e_j would leave float range): the
+    //     output sum F' = sum_j acc_j e_j (tensor memory) and the softmax sum L' = sum_j l_j e_j
+    //     (shared memory) give O = F' v_scale / (255 L'), the blockwise online softmax's result.
+    //   * The fold of block j (F' += acc_j e_j, L' += l_j e_j) is done by block j's group after
+    //     P.V(j); P.V(j + 1) waits for it (one accumulator), so the folds, and every update of
+    //     F', L' and m_ref, run in block order.
+    const int grp = (warp - 4) >> 2, w4 = warp & 3;
     const int r = w4 * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(w4 * 32) << 16;
-    const uint32_t aS = tmem + lane_base + C::tS(q);
-    const uint32_t aP = tmem + lane_base + C::tP(q);
-    const uint32_t aO0 = tmem + lane_base + C::tO(q, 0);
-    const uint32_t aO1 = tmem + lane_base + C::tO(q, 1);
-    const uint32_t aF = tmem + lane_base + C::tF(q);  // unused when F is in shared memory
-    // Fast path: full key blocks, no debug output, aligned dense rows, rel-pos table in shared
-    // memory with the class tokens handled by the zero padding.
-    const bool fast_ok = (p.dbg_logits == nullptr) &&
-                         (BK != BA_BIAS_DENSE || ((N & 3) == 0 && (p.bias.batch_stride & 3) == 0)) &&
-                         (!is_relpos(BK) || p.bias.n_prefix == 0 || tab_mode == 2);
+    const uint32_t aAcc = tmem + lane_base + C::tAcc(0);
+    const uint32_t aF = tmem + lane_base + C::tF(0);
+    float* s_m = reinterpret_cast<float*>(smem + C::offX);  // [2][BM] m_j by block parity
+    // [BM] (L', m_ref) of each row, stored as one 8-byte pair so that a reader outside the fold
+    // chain sees a consistent pair.
+    float2* s_Lm = reinterpret_cast<float2*>(s_m + 2 * BM);
+    uint64_t* mch = &bars[Bar::mchain(w4)];
+    // Share of the error bar one changed code may take in a row that is not checked.
+    constexpr float kCheckTau = 2.0e-4f;
+    constexpr float kTieBand = 0.5f - 2.5e-4f;
     bool alive = true;
-    // Accumulator that P.V of the current block adds into (tile-uniform): every item starts on
-    // the other one, as the MMA thread does.
-    int cur = 1;
     float mu_q_next = 0.0f, mu_k_next = 0.0f;  // mu of the item about to start (loaded one item ahead)
     int n0 = 0;  // index, counted across items, of the item's first key block
     for (int it = 0; it < n_items && alive; ++it, n0 += T) {
-    int64_t bh;
-    int q0;
-    item_at(by_head, it, p.H, nqb, BM * NQ, bh, q0);
-    const int64_t b = bh / p.H, h = bh - b * p.H;
-    const int i = q0 + q * BM + r;
-    const bool row_ok = i < N;
-    const int ic = row_ok ? i : N - 1;  // rows past N read the bias of row N-1 (never stored)
-    if (it == 0) {
-      mu_q_next = p.mu_q[bh];
-      mu_k_next = p.mu_k[bh];
-    }
-    const float alpha = __fmul_rn(__fmul_rn(p.softmax_scale, mu_q_next), mu_k_next);
-    const float2 alpha2 = make_float2(alpha, alpha);
+      int64_t bh;
+      int q0;
+      item_at(by_head, it, p.H, nqb, BM, bh, q0);
+      const int64_t b = bh / p.H, h = bh - b * p.H;
+      const int i = q0 + r;
+      const bool row_ok = i < N;
+      const int ic = row_ok ? i : N - 1;  // rows past N read the bias of row N-1 (never stored)
+      if (it == 0) {
+        mu_q_next = p.mu_q[bh];
+        mu_k_next = p.mu_k[bh];
+      }
+      const float alpha = __fmul_rn(__fmul_rn(p.softmax_scale, mu_q_next), mu_k_next);
+      const float2 alpha2 = make_float2(alpha, alpha);
+      // The head's largest |V| (127 times its largest channel scale) bounds what one changed
+      // code can move an output by: |v| / (255 l). Blocks of rows whose softmax sum l is below
+      // l_check = max|V| / (255 tau) get their near-tie codes recomputed exactly.
+      float vmax = 0.0f;
+#pragma unroll
+      for (int k = 0; k < (DP + 31) / 32; ++k)
+        if (32 * k + lane < d) vmax = fmaxf(vmax, p.v_scale[bh * d + 32 * k + lane]);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
+      const float l_check = (127.0f * vmax) / (255.0f * kCheckTau);
 
-    // Bias addressing. Dense: this row of [H][N][N]. Rel-pos: b_ij = tab[a_i - koff_j] with
-    // tab the head's table (staged in shared memory when it fits, followed by zeros that
-    // class-token rows and keys index into), koff_j kept as byte offsets.
-    const float* brow = nullptr;
-    const float* gtab = nullptr;
-    int a_i = 0;
-    if (BK == BA_BIAS_DENSE) brow = p.bias.data + b * p.bias.batch_stride + (h * N + ic) * N;
-    if (is_relpos(BK)) {
-      const int W2 = 2 * p.bias.table_w - 1;
-      gtab = p.bias.data + h * static_cast<int64_t>(2 * p.bias.table_h - 1) * W2;
-      if (ic >= p.bias.n_prefix) {
-        const int ti = ic - p.bias.n_prefix;
-        const int yi = ti / p.bias.grid_w;
-        a_i = (yi + p.bias.table_h - 1) * W2 + (ti - yi * p.bias.grid_w) + p.bias.table_w - 1;
-      } else {
-        a_i = (tab_mode == 2) ? tsize + kmax : -1;  // class-token row: the zeros (or the general path)
-      }
-    }
-    const uint32_t tb = smem_u32(stab) + 4u * static_cast<uint32_t>(a_i);  // this row's table base
-    const float* grow = gtab + a_i;  // this row's base in a table left in global memory
-
-    float m = -CUDART_INF_F, l = 0.0f;
-    // Whether F holds anything yet, and how many blocks the current accumulator holds.
-    int nblk = 1;
-    bool f_valid = false;
-    cur ^= 1;
-
-    for (int t = 0; t < T && alive; ++t) {
-      const int n = n0 + t;
-      const int st = n % S;
-      const int nk = min(BN, N - t * BN);
-      // 32-key chunks that hold keys of this block. The P codes of the chunks past them are
-      // left as they are: they multiply V rows past N, which the V copy fills with zeros.
-      const int nch = (nk + 31) >> 5;
-      if (is_relpos(BK) && !wait_warp(&bars[Bar::kvfull(st)], (n / S) & 1, abort_flag)) {
-        alive = false;
-        break;
-      }
-      if (!wait_warp(&bars[Bar::sfull(q)], n & 1, abort_flag)) {
-        alive = false;
-        break;
-      }
-      tc_fence_after();
-      const uint32_t ko_s = smem_u32(koff + st * BN);
-
-      // Pass 1: s = alpha * x + b written back over S in TMEM; block max. The next 32-column
-      // block is loaded from TMEM while this one is computed.
-      float mx[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
-      // The fast path also takes a partial last block (keys past N are masked to -inf after
-      // the fact; their rel-pos offsets point at valid entries), except for dense bias rows,
-      // which end at N.
-      const bool fast = fast_ok && (nk == BN || BK != BA_BIAS_DENSE);
-      {
-        // One copy of the block body (a small hot loop stays in the instruction cache; the
-        // other softmax warps of the SM cover the TMEM load latency).
-#pragma unroll 1
-        for (int c = 0; c < nch; ++c) {
-          uint32_t x[32];
-          tmem_ld32(aS + 32 * c, x);
-          tmem_ld_wait();
-          reg_fence32(x);
-          if (fast) {
-            if (nk == BN)
-              fast_block<BK, false>(x, c, nk, alpha2, brow + t * BN, ko_s, tb, grow, tab_mode, mx);
-            else
-              fast_block<BK, true>(x, c, nk, alpha2, brow + t * BN, ko_s, tb, grow, tab_mode, mx);
-          } else {
-            // General path: a partial last block, class tokens without zero padding,
-            // unaligned dense rows, a table in global memory, or the debug logits.
-#pragma unroll
-            for (int u = 0; u < 32; ++u) {
-              const int j = 32 * c + u;
-              float sv = -CUDART_INF_F;
-              if (j < nk) {
-                const float xf = __uint_as_float(x[u]);
-                float bias = 0.0f;
-                if (BK == BA_BIAS_DENSE) bias = __ldg(brow + t * BN + j);
-                if (is_relpos(BK)) {
-                  const int kj = lds_s32(ko_s + 4u * j) >> 2;
-                  if (a_i >= 0 && kj >= 0)
-                    bias = (tab_mode != 0) ? lds_f32(smem_u32(stab) + 4u * static_cast<uint32_t>(a_i - kj))
-                                           : __ldg(gtab + (a_i - kj));
-                }
-                sv = __fmaf_rn(alpha, xf, bias);
-                if (p.dbg_logits != nullptr && row_ok)
-                  p.dbg_logits[(bh * N + i) * N + t * BN + j] = __float2int_rn(xf);
-              }
-              mx[u & 3] = fmaxf(mx[u & 3], sv);
-              x[u] = __float_as_uint(sv);
-            }
-          }
-          tmem_st32(aS + 32 * c, x);
-        }
-      }
-      const float m_new = fmaxf(m, fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])));
-      tmem_st_wait();
-
-      // Pass 2: P~ = 2^((s - m) log2 e) (masked keys hold s = -inf: P~ = 0), row sum, u8 codes
-      // -> TMEM columns 0..31 (their s values were read in the first step of this pass).
-      const float2 negm2 = make_float2(-m_new, -m_new);
-      const float2 log2e2 = make_float2(kLog2e, kLog2e);
-      const float2 c255 = make_float2(255.0f, 255.0f);
-      const float2 magic2 = make_float2(12582912.0f, 12582912.0f);
-      float2 lt2[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
-      {
-#pragma unroll 1
-        for (int c = 0; c < nch; ++c) {
-          uint32_t x[32];
-          tmem_ld32(aS + 32 * c, x);
-          tmem_ld_wait();
-          reg_fence32(x);
-          uint32_t pk[8];
-#pragma unroll
-          for (int w = 0; w < 8; ++w) {
-            uint32_t y[4];
-#pragma unroll
-            for (int e2 = 0; e2 < 2; ++e2) {
-              const int u = 4 * w + 2 * e2;
-              // s - m first (exact near the max), then the scale to base 2.
-              const float2 t2 = __fmul2_rn(
-                  __fadd2_rn(make_float2(__uint_as_float(x[u]), __uint_as_float(x[u + 1])), negm2), log2e2);
-              const float2 p2 = ((kPolyPairs >> (2 * w + e2)) & 1u) ? exp2_poly2(t2)
-                                                                    : make_float2(ex2_approx(t2.x), ex2_approx(t2.y));
-              lt2[e2] = __fadd2_rn(lt2[e2], p2);
-              // 255 P~ + 1.5 * 2^23: one rounding to the nearest integer (ties to even); the
-              // integer sits in the low byte of the result (P~ <= 1).
-              const float2 y2 = __ffma2_rn(p2, c255, magic2);
-              y[2 * e2] = __float_as_uint(y2.x);
-              y[2 * e2 + 1] = __float_as_uint(y2.y);
-            }
-            pk[w] = __byte_perm(__byte_perm(y[0], y[1], 0x0040), __byte_perm(y[2], y[3], 0x0040), 0x5410);
-          }
-          tmem_st8(aP + 8 * c, pk);
-        }
-      }
-      const float lt = (lt2[0].x + lt2[0].y) + (lt2[1].x + lt2[1].y);
-      // Rescale factor of the row's earlier blocks: exactly 1 while its max is unchanged.
-      const float ct = (m == -CUDART_INF_F) ? 0.0f : (m_new > m ? ex2_approx((m - m_new) * kLog2e) : 1.0f);
-      l = l * ct + lt;
-      // Vote (per warp) whether a row raised its max; the MMA thread reads the votes of the
-      // tile's four warps after their p_full arrivals.
-      const bool rose = __any_sync(0xffffffffu, t > 0 && m_new > m);
-      if (lane == 0) votes[((n & 1) * NQ + q) * 4 + w4] = rose ? 1u : 0u;
-      m = m_new;
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[Bar::pfull(q)]);
-      if (t == 0) continue;
-      // While the MMAs of the next block run: if any row of the tile raised its max, P.V of
-      // this block goes to the other accumulator, and the old one is folded into F with this
-      // row's factor (1 for rows whose max did not rise).
-      if (!wait_warp(&bars[Bar::pfull(q)], n & 1, abort_flag)) {
-        alive = false;
-        break;
-      }
-      const volatile uint32_t* vt = votes + ((n & 1) * NQ + q) * 4;
-      if ((vt[0] | vt[1] | vt[2] | vt[3]) != 0u) {
-        fold_rest<C, 0>(cur ? aO1 : aO0, aF, sF + q * BM + r, make_float2(ct, ct), !f_valid, nblk == 1);
-        if (!C::kFSmem) tmem_st_wait();
-        cur ^= 1;
-        f_valid = true;
-        nblk = 1;
-      } else {
-        ++nblk;
-      }
-    }
-
-    // This item's V scales / 255 (lane l of every warp holds channels l, l + 32, ..., read by
-    // shuffles in the epilogue) and the next item's mu, loaded while the last P.V runs.
-    float scv[(DP + 31) / 32];
-#pragma unroll
-    for (int k = 0; k < (DP + 31) / 32; ++k)
-      scv[k] = (32 * k + lane < d) ? p.v_scale[bh * d + 32 * k + lane] * (1.0f / 255.0f) : 0.0f;
-    if (it + 1 < n_items) {
-      int64_t nbh;
-      int nq0;
-      item_at(by_head, it + 1, p.H, nqb, BM * NQ, nbh, nq0);
-      mu_q_next = p.mu_q[nbh];
-      mu_k_next = p.mu_k[nbh];
-    }
-    if (alive && wait_warp(&bars[Bar::odone(q)], it & 1, abort_flag)) {
-      tc_fence_after();
-      const float inv_l = 1.0f / l;
-      // Rows whose byte length is a multiple of 16 are written with 16-byte stores (each
-      // thread owns one row); other shapes fall back to element stores.
-      const int esz = (p.o_dt == BA_F32) ? 4 : 2;
-      const bool vec = ((d * esz) & 15) == 0;
-      char* orow = reinterpret_cast<char*>(p.o) + ((bh * N + i) * d) * esz;
-      const uint32_t aO = cur ? aO1 : aO0;
-      const float4* fr = sF + q * BM + r;
-#pragma unroll 1
-      for (int cc = 0; cc < DP / 16; ++cc) {
-        uint32_t a[16], fb[16];
-        tmem_ld16(aO + 16 * cc, a);
-        if constexpr (!C::kFSmem) tmem_ld16(aF + 16 * cc, fb);  // read even before the first fold
-        tmem_ld_wait();
-        reg_fence16(a);
-        if constexpr (!C::kFSmem) reg_fence16(fb);
-        float val[16];
-        // Scales of channels 16 cc .. 16 cc + 15: held by lanes 16 (cc & 1) ... of register cc / 2.
-        float sreg = scv[0];
-#pragma unroll
-        for (int k = 1; k < (DP + 31) / 32; ++k)
-          if (cc >= 2 * k) sreg = scv[k];  // constant comparisons keep scv in registers
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          float fv;
-          if constexpr (C::kFSmem) {
-            const float4 v4 = fr[(4 * cc + (e >> 2)) * (NQ * BM)];
-            fv = (e & 3) == 0 ? v4.x : ((e & 3) == 1 ? v4.y : ((e & 3) == 2 ? v4.z : v4.w));
-          } else {
-            fv = __uint_as_float(fb[e]);
-          }
-          if (!f_valid) fv = 0.0f;
-          const float sc = __shfl_sync(0xffffffffu, sreg, 16 * (cc & 1) + e);
-          val[e] = (fv + __int2float_rn(static_cast<int>(a[e]))) * sc * inv_l;
-        }
-        if (!row_ok) continue;
-        if (vec && 16 * cc + 16 <= d) {
-          if (p.o_dt == BA_F32) {
-#pragma unroll
-            for (int k4 = 0; k4 < 4; ++k4)
-              reinterpret_cast<float4*>(orow + (16 * cc + 4 * k4) * 4)[0] =
-                  make_float4(val[4 * k4], val[4 * k4 + 1], val[4 * k4 + 2], val[4 * k4 + 3]);
-          } else {
-            uint32_t h[8];
-#pragma unroll
-            for (int k2 = 0; k2 < 8; ++k2) {
-              if (p.o_dt == BA_F16) {
-                const __half2 v = __floats2half2_rn(val[2 * k2], val[2 * k2 + 1]);
-                h[k2] = *reinterpret_cast<const uint32_t*>(&v);
-              } else {
-                const __nv_bfloat162 v = __floats2bfloat162_rn(val[2 * k2], val[2 * k2 + 1]);
-                h[k2] = *reinterpret_cast<const uint32_t*>(&v);
-              }
-            }
-            reinterpret_cast<uint4*>(orow + 16 * cc * 2)[0] = make_uint4(h[0], h[1], h[2], h[3]);
-            reinterpret_cast<uint4*>(orow + 16 * cc * 2)[1] = make_uint4(h[4], h[5], h[6], h[7]);
-          }
+      // Bias addressing. Dense: this row of [H][N][N]. General rel-pos: b_ij = tab[a_i - koff_j]
+      // (table staged in shared memory when it fits, followed by zeros that class-token rows and
+      // keys index into). Window: b_ij = window[A_i - K_c - u].
+      const float* brow = nullptr;
+      const float* gtab = nullptr;
+      int a_i = 0;
+      if constexpr (BK == kBiasDense) brow = p.bias.data + b * p.bias.batch_stride + (h * N + ic) * N;
+      if constexpr (is_relpos_general(BK)) {
+        const int W2 = 2 * p.bias.table_w - 1;
+        gtab = p.bias.data + h * static_cast<int64_t>(2 * p.bias.table_h - 1) * W2;
+        if (ic >= p.bias.n_prefix) {
+          const int ti = ic - p.bias.n_prefix;
+          const int yi = ti / p.bias.grid_w;
+          a_i = (yi + p.bias.table_h - 1) * W2 + (ti - yi * p.bias.grid_w) + p.bias.table_w - 1;
         } else {
-#pragma unroll
-          for (int e = 0; e < 16; ++e)
-            if (16 * cc + e < d) store_out(p.o, (bh * N + i) * d + 16 * cc + e, val[e], p.o_dt);
+          a_i = (tab_mode == 2) ? tsize + kmax : -1;  // class-token row: the zeros (or the per-key test)
         }
       }
-    }
-    }
-  }
-
-  // ------------------------------------------------------------ teardown
-  tc_fence_before();
-  named_barrier_sync(1, C::kThreads);
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem, C::kTmemCols);
-  }
-}
-
-// The same forward with one work item per CTA (no persistent loop): used for heads wider than
-// 80 channels (one 128-row tile per CTA, F in tensor memory), where it measured faster than the
-// persistent kernel on B200.
-template <int DP, int BK, int NQ_>
-__global__ void __launch_bounds__(Cfg<DP, NQ_>::kThreads, Cfg<DP, NQ_>::kCtasPerSm)
-    attn_tc_single_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmap_v, int tab_mode, int tsize,
-                   int kmax) {
-  using C = Cfg<DP, NQ_>;
-  constexpr int NQ = C::NQ, DQ = C::DQ, S = C::kStages;
-  using Bar = Bars<S, NQ>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem + C::offQ;
-  uint8_t* sK = smem + C::offK;
-  uint8_t* sV = smem + C::offV;
-  int* koff = reinterpret_cast<int*>(smem + C::offKoff);
-  float* sscale = reinterpret_cast<float*>(smem + C::offScale);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::offBar);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::offMisc);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::offMisc + 4);
-  // Per block parity, tile and softmax warp: whether a row of that warp raised its max.
-  uint32_t* votes = reinterpret_cast<uint32_t*>(smem + C::offVotes);
-  float4* sF = reinterpret_cast<float4*>(smem + C::offF);  // [DP/4][NQ*128]
-  // Rel-pos table of this CTA's head, staged when it fits: tab_mode 1 = table only,
-  // 2 = table followed by 2*tsize zeros (targets of prefix rows and prefix keys).
-  float* stab = reinterpret_cast<float*>(smem + C::kTabOff);
-
-  const int N = p.N, d = p.d;
-  const int ctas_per_bh = static_cast<int>(ceil_div(N, BM * NQ));
-  const int64_t bh = blockIdx.x / ctas_per_bh;
-  const int q0 = static_cast<int>(blockIdx.x - bh * ctas_per_bh) * BM * NQ;
-  const int64_t b = bh / p.H, h = bh - b * p.H;
-  const int T = static_cast<int>(ceil_div(N, BN));
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-  if (threadIdx.x == 0) {
-    for (int st = 0; st < C::kStages; ++st) {
-      // kv_full: the V copy's expect_tx arrival + warp 0 (key offsets) + the two expanding warps.
-      mbar_init(&bars[Bar::kvfull(st)], 4);
-      mbar_init(&bars[Bar::kvempty(st)], 1);
-    }
-    mbar_init(&bars[Bar::qfull()], 2);
-    mbar_init(&bars[Bar::drain()], 1);
-    for (int q = 0; q < NQ; ++q) {
-      mbar_init(&bars[Bar::sfull(q)], 1);
-      mbar_init(&bars[Bar::pfull(q)], 4);
-      mbar_init(&bars[Bar::odone(q)], 1);
-    }
-    *abort_flag = 0;
-    mbar_fence_init();
-    fence_proxy_async_smem();
-    tma_prefetch_desc(&tmap_v);
-  }
-  // Warps 2 and 3 load the sign rows of their Q rows and of key block 0 before the setup barrier,
-  // so the loads overlap the setup.
-  const uint4 zero4 = make_uint4(0u, 0u, 0u, 0u);
-  uint4 pre_q[NQ][2], pre_k[2];
-  if (warp == 2 || warp == 3) {
-    const int half = warp - 2;
-    const uint4* qrows = reinterpret_cast<const uint4*>(p.bits_q) + bh * N;
-    const uint4* krows = reinterpret_cast<const uint4*>(p.bits_k) + bh * N;
-#pragma unroll
-    for (int q = 0; q < NQ; ++q)
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int row = q0 + q * BM + 64 * half + lane + 32 * u;
-        pre_q[q][u] = row < N ? __ldg(qrows + row) : zero4;
+      int A_i = 0;
+      if constexpr (BK == kRelWindow) {
+        const int yi = ic / p.bias.grid_w;
+        A_i = yi * win_stride + (ic - yi * p.bias.grid_w);
       }
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int row = 64 * half + lane + 32 * u;
-      pre_k[u] = row < N ? __ldg(krows + row) : zero4;
-    }
-  }
-  if (threadIdx.x < 128)
-    sscale[threadIdx.x] = (threadIdx.x < d) ? p.v_scale[bh * d + threadIdx.x] * (1.0f / 255.0f) : 0.0f;
-  if (is_relpos(BK) && tab_mode != 0) {
-    const float* src = p.bias.data + h * static_cast<int64_t>(tsize);
-    const int n = (tab_mode == 2) ? 3 * tsize : tsize;
-    for (int e = threadIdx.x; e < n; e += C::kThreads) stab[e] = (e < tsize) ? __ldg(src + e) : 0.0f;
-  }
-  if (warp == 1) {
-    tmem_alloc(tmem_slot, C::kTmemCols);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
+      const bool dense_vec = BK == kBiasDense && (N & 3) == 0 && (p.bias.batch_stride & 3) == 0;
+      // (L', m_ref) after this group's last fold in the item (own registers: the check decision
+      // below must not depend on when the other group's fold lands, or results would vary
+      // from run to run); L' = 0 before the group's first fold of the item.
+      float own_L = 0.0f, own_mref = 0.0f;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer: V blocks, key offsets
-    const int W2 = 2 * p.bias.table_w - 1;
-    int issued = 0;
-    for (int t = 0; t < T; ++t) {
-      const int st = t % S;
-      if (t >= S && !wait_warp(&bars[Bar::kvempty(st)], ((t / S) - 1) & 1, abort_flag)) break;
-      issued = t + 1;
-      if (lane == 0) {
-        mbar_arrive_expect_tx(&bars[Bar::kvfull(st)], C::kVBytes);
-        tma_load_4d(sV + st * C::kVBytes, &tmap_v, &bars[Bar::kvfull(st)], 0, t * BN, 0, static_cast<int>(bh));
-      }
-      if (is_relpos(BK)) {
-#pragma unroll
-        for (int u = 0; u < BN / 32; ++u) {
-          const int j = lane + 32 * u, tok = t * BN + j;
-          // Keys past N read a valid entry (their P is masked); prefix keys read the zeros
-          // after the staged table (or are marked -1 for the general path).
-          int v = (tab_mode == 2) ? -tsize : -1;
-          if (tok >= N) {
-            v = 0;
-          } else if (tok >= p.bias.n_prefix) {
-            const int tj = tok - p.bias.n_prefix;
-            const int yj = tj / p.bias.grid_w;
-            v = yj * W2 + (tj - yj * p.bias.grid_w);
+      for (int t = grp ^ (n0 & 1); t < T && alive; t += 2) {
+        const int n = n0 + t;
+        const int st = n % S;
+        const int j0 = t * BN;
+        const int nk = min(BN, N - j0);  // valid keys of this block
+        const uint32_t aS = tmem + lane_base + C::tS(0, n & 1);
+        if constexpr (BK == kRelWindow || is_relpos_general(BK)) {
+          if (!wait_warp(&bars[Bar::kvfull(st)], (n / S) & 1, abort_flag)) {
+            alive = false;
+            break;
           }
-          koff[st * BN + j] = 4 * v;  // byte offset into the staged table
         }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[Bar::kvfull(st)]);
-    }
-    // Leave no TMA copy in flight: wait (bounded, even after an abort) for the stages this
-    // warp filled last.
-    for (int t = (issued > S ? issued - S : 0); t < issued; ++t)
-      wait_bounded(&bars[Bar::kvfull(t % S)], (t / S) & 1, abort_flag, false);
-  } else if (warp == 2 || warp == 3) {
-    // ------------------------------------------------------------ producer: sign expansion
-    // Warp 2 expands rows 0..63 and warp 3 rows 64..127 of every Q tile and K block. The
-    // sign rows of the next block are loaded into registers before this block is written.
-    const int half = warp - 2;
-    const uint4* krows = reinterpret_cast<const uint4*>(p.bits_k) + bh * N;
-#pragma unroll
-    for (int q = 0; q < NQ; ++q)
-#pragma unroll
-      for (int u = 0; u < 2; ++u)
-        expand_row<DQ>(sQ + q * C::kQBytes, pre_q[q][u], q0 + q * BM + 64 * half + lane + 32 * u < N,
-                       64 * half + lane + 32 * u, d);
-    fence_proxy_async_smem();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&bars[Bar::qfull()]);
-    uint4 nb[2] = {pre_k[0], pre_k[1]};
-    for (int t = 0; t < T; ++t) {
-      const int st = t % S;
-      const uint4 cb[2] = {nb[0], nb[1]};
-      if (t + 1 < T) {
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int row = (t + 1) * BN + 64 * half + lane + 32 * u;
-          nb[u] = row < N ? __ldg(krows + row) : zero4;
+        if (!wait_warp(&bars[Bar::sfull(0, n & 1)], (n >> 1) & 1, abort_flag)) {
+          alive = false;
+          break;
         }
-      }
-      if (t >= S && !wait_warp(&bars[Bar::kvempty(st)], ((t / S) - 1) & 1, abort_flag)) break;
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int r = 64 * half + lane + 32 * u;
-        expand_row<DQ>(sK + st * C::kKBytes, cb[u], t * BN + r < N, r, d);
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[Bar::kvfull(st)]);
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t idesc_qk = (1u << 4) | (0u << 7) | (0u << 10) | (static_cast<uint32_t>(BN >> 3) << 17) |
-                                (static_cast<uint32_t>(BM >> 4) << 24);
-      const uint32_t idesc_pv = (2u << 4) | (0u << 7) | (1u << 10) | (1u << 16) |
-                                (static_cast<uint32_t>(DP >> 3) << 17) | (static_cast<uint32_t>(BM >> 4) << 24);
-      if (wait_bounded(&bars[Bar::qfull()], 0, abort_flag)) {
         tc_fence_after();
-        bool ok = true;
-        uint32_t cur_acc = 0;  // bit q: the accumulator P.V of tile q adds into
-        for (int t = 0; t <= T && ok; ++t) {
-          for (int q = 0; q < NQ && ok; ++q) {
-            // P.V of the previous block first (it needs no new operands), then QK of this
-            // block into the same S columns (issue order keeps P read before S is rewritten).
-            if (t > 0) {
-              if (!wait_bounded(&bars[Bar::pfull(q)], (t - 1) & 1, abort_flag)) {
-                ok = false;
-                break;
-              }
-              tc_fence_after();
-              // Block 0 starts accumulator 0. Later blocks switch to the other accumulator
-              // (overwriting it) when a row of the tile raised its max: the softmax warps'
-              // votes, written before their p_full arrivals.
-              bool fresh = (t == 1);
-              if (t > 1) {
-                const volatile uint32_t* vt = votes + (((t - 1) & 1) * NQ + q) * 4;
-                if ((vt[0] | vt[1] | vt[2] | vt[3]) != 0u) {
-                  cur_acc ^= 1u << q;
-                  fresh = true;
-                }
-              }
-              const uint32_t acc = tmem + C::tO(q, (cur_acc >> q) & 1u);
-              const uint32_t vbase = smem_u32(sV + ((t - 1) % S) * C::kVBytes);
+
+        // ---- pass 1: s = alpha x + b over four 32-key chunks (the next chunk's load in flight
+        // while this one is formed), written back over S; the block maximum.
+        float mx[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
+        auto pass1 = [&](auto masked) {
+          constexpr bool MASK = decltype(masked)::value;
+          // A rolled loop over pairs of chunks (two copies of the chunk body, not four, keep the
+          // hot code in the instruction cache); buffers xa / xb alternate, the next chunk's load
+          // in flight while this one is worked on.
+          uint32_t xa[32], xb[32];
+          tmem_ld_cols<32>(aS, xa);
+#pragma unroll 1
+          for (int cp = 0; cp < BN / 64; ++cp)
 #pragma unroll
-              for (int kk = 0; kk < BN / 32; ++kk)
-                mma_i8_ts(acc, tmem + C::tP(q) + 8 * kk, smem_desc(vbase + 512 * kk, 128, 2048), idesc_pv,
-                          (fresh && kk == 0) ? 0u : 1u);
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const int c = 2 * cp + h2;
+            uint32_t* x = h2 ? xb : xa;
+            uint32_t* xn = h2 ? xa : xb;
+            tmem_ld_wait();
+            reg_fence_cols<32>(x);
+            if (c + 1 < BN / 32) tmem_ld_cols<32>(aS + 32 * (c + 1), xn);
+            const int jc = j0 + 32 * c;  // first key of this chunk
+            if (p.dbg_logits != nullptr && row_ok) {
+#pragma unroll
+              for (int u = 0; u < 32; ++u)
+                if (32 * c + u < nk) p.dbg_logits[(bh * N + i) * N + jc + u] = __float2int_rn(__uint_as_float(x[u]));
             }
-            if (t < T) {
-              if (q == 0) {
-                if (!wait_bounded(&bars[Bar::kvfull(t % S)], (t / S) & 1, abort_flag)) {
-                  ok = false;
-                  break;
-                }
-                tc_fence_after();
-              }
-              const uint32_t qb = smem_u32(sQ + q * C::kQBytes), kb = smem_u32(sK + (t % S) * C::kKBytes);
+            const float* wrow = nullptr;
+            (void)wrow;
+            if constexpr (BK == kRelWindow) {
+              // Every chunk lies in one grid row (grid width a multiple of 32, N = grid size), so
+              // its 32 biases are a descending run of the window. Chunks past N are masked.
+              const int kc = jc < N ? swink[st * 4 + c] : A_i - 31;
+              wrow = swin + st * kWinFloats + (A_i - kc);
+            }
 #pragma unroll
-              for (int kk = 0; kk < DQ / 32; ++kk)
-                mma_f8f6f4_ss(tmem + C::tS(q), smem_desc(qb + kk * 4096, 2048, 128),
-                              smem_desc(kb + kk * 4096, 2048, 128), idesc_qk, kk > 0 ? 1u : 0u);
-              tc_commit(&bars[Bar::sfull(q)]);
-            } else {
-              tc_commit(&bars[Bar::odone(q)]);
+            for (int g8 = 0; g8 < 4; ++g8) {
+              float bv[8];
+              const int j8 = jc + 8 * g8;
+              (void)j8;
+              if constexpr (BK == kBiasNone) {
+#pragma unroll
+                for (int u = 0; u < 8; ++u) bv[u] = 0.0f;
+              } else if constexpr (BK == kBiasDense) {
+                if (dense_vec && j8 + 8 <= N) {
+                  const float4 v0 = __ldg(reinterpret_cast<const float4*>(brow + j8));
+                  const float4 v1 = __ldg(reinterpret_cast<const float4*>(brow + j8) + 1);
+                  bv[0] = v0.x; bv[1] = v0.y; bv[2] = v0.z; bv[3] = v0.w;
+                  bv[4] = v1.x; bv[5] = v1.y; bv[6] = v1.z; bv[7] = v1.w;
+                } else {
+#pragma unroll
+                  for (int u = 0; u < 8; ++u) bv[u] = (j8 + u < N) ? __ldg(brow + j8 + u) : 0.0f;
+                }
+              } else if constexpr (BK == kRelWindow) {
+#pragma unroll
+                for (int u = 0; u < 8; ++u) bv[u] = wrow[-(8 * g8 + u)];
+              } else {
+                const uint32_t ko = smem_u32(koff + st * BN + 32 * c + 8 * g8);
+                if (BK == kRelSmem && tab_mode == 2) {
+                  const uint32_t tb = smem_u32(stab) + 4u * static_cast<uint32_t>(a_i);
+                  const int4 o0 = lds_s32x4(ko), o1 = lds_s32x4(ko + 16u);
+                  bv[0] = lds_f32(tb - 4u * o0.x); bv[1] = lds_f32(tb - 4u * o0.y);
+                  bv[2] = lds_f32(tb - 4u * o0.z); bv[3] = lds_f32(tb - 4u * o0.w);
+                  bv[4] = lds_f32(tb - 4u * o1.x); bv[5] = lds_f32(tb - 4u * o1.y);
+                  bv[6] = lds_f32(tb - 4u * o1.z); bv[7] = lds_f32(tb - 4u * o1.w);
+                } else {
+#pragma unroll
+                  for (int u = 0; u < 8; ++u) {
+                    const int kj = lds_s32(ko + 4u * u);
+                    float bias = 0.0f;
+                    if (a_i >= 0 && kj >= 0)
+                      bias = (BK == kRelSmem) ? lds_f32(smem_u32(stab) + 4u * static_cast<uint32_t>(a_i - kj))
+                                              : __ldg(gtab + (a_i - kj));
+                    bv[u] = bias;
+                  }
+                }
+              }
+#pragma unroll
+              for (int u = 0; u < 8; u += 2) {
+                const int k = 8 * g8 + u;
+                float2 s2;
+                if constexpr (BK == kBiasNone)
+                  s2 = __fmul2_rn(alpha2, make_float2(__uint_as_float(x[k]), __uint_as_float(x[k + 1])));
+                else
+                  s2 = __ffma2_rn(alpha2, make_float2(__uint_as_float(x[k]), __uint_as_float(x[k + 1])),
+                                  make_float2(bv[u], bv[u + 1]));
+                if (MASK) {
+                  if (32 * c + k >= nk) s2.x = -CUDART_INF_F;
+                  if (32 * c + k + 1 >= nk) s2.y = -CUDART_INF_F;
+                }
+                x[k] = __float_as_uint(s2.x);
+                x[k + 1] = __float_as_uint(s2.y);
+                mx[(u >> 1) & 3] = fmax3(mx[(u >> 1) & 3], s2.x, s2.y);
+              }
+            }
+            tmem_st_cols<32>(aS + 32 * c, x);
+          }
+        };
+        if (nk < BN)
+          pass1(std::true_type{});
+        else
+          pass1(std::false_type{});
+        const float bmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+        tmem_st_wait();  // s is in S before pass 2 reads it back
+
+        // ---- the running maximum: m_{n-1} from the other group (block n - 1), then m_n out
+        float m_prev = -CUDART_INF_F;
+        if (n > 0) {
+          if (!wait_warp(mch, (n - 1) & 1, abort_flag)) {
+            alive = false;
+            break;
+          }
+          if (t > 0) m_prev = s_m[((n - 1) & 1) * BM + r];
+        }
+        const float m_new = fmaxf(m_prev, bmax);
+        s_m[(n & 1) * BM + r] = m_new;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(mch);
+        // Rows whose softmax sum so far is small get the exact near-tie check. The sum is taken
+        // as of this group's own last fold (an underestimate of the row's true sum).
+        const float l_so_far = own_L > 0.0f ? own_L * ex2_approx((own_mref - m_new) * kLog2e) : 0.0f;
+        const bool check = p.p_check_all || __any_sync(0xffffffffu, l_so_far + 1.0f < l_check);
+
+        // ---- pass 2: P~ = 2^((s - m) log2 e), row sum, 8-bit codes (masked keys: s = -inf,
+        // P~ = 0) per 32-key chunk, near-tie codes of each 16-key group settled in place; the
+        // codes go to columns 8c .. 8c + 7 of the S buffer (keys 0..31 of S, read already).
+        const float2 negm2 = make_float2(-m_new, -m_new);
+        const float2 log2e2 = make_float2(kLog2e, kLog2e);
+        const float2 c255 = make_float2(255.0f, 255.0f);
+        const float2 magic2 = make_float2(kMagic, kMagic);
+        float2 lt2[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
+        auto pass2 = [&](auto checked) {
+          constexpr bool CHECK = decltype(checked)::value;
+          // A rolled loop over pairs of chunks (two copies of the chunk body, not four, keep the
+          // hot code in the instruction cache); buffers xa / xb alternate, the next chunk's load
+          // in flight while this one is worked on.
+          uint32_t xa[32], xb[32];
+          tmem_ld_cols<32>(aS, xa);
+#pragma unroll 1
+          for (int cp = 0; cp < BN / 64; ++cp)
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const int c = 2 * cp + h2;
+            uint32_t* x = h2 ? xb : xa;
+            uint32_t* xn = h2 ? xa : xb;
+            tmem_ld_wait();
+            reg_fence_cols<32>(x);
+            if (c + 1 < BN / 32) tmem_ld_cols<32>(aS + 32 * (c + 1), xn);
+            uint32_t pk[8];
+#pragma unroll
+            for (int g4 = 0; g4 < 2; ++g4) {
+              float rmx = 0.0f;
+#pragma unroll
+              for (int w = 4 * g4; w < 4 * g4 + 4; ++w) {
+                uint32_t y[4];
+#pragma unroll
+                for (int e2 = 0; e2 < 2; ++e2) {
+                  const int k = 4 * w + 2 * e2;
+                  // s - m first (exact near the maximum), then the scale to base 2.
+                  const float2 t2 = __fmul2_rn(
+                      __fadd2_rn(make_float2(__uint_as_float(x[k]), __uint_as_float(x[k + 1])), negm2), log2e2);
+                  const float2 p2 = make_float2(ex2_approx(t2.x), ex2_approx(t2.y));
+                  lt2[e2] = __fadd2_rn(lt2[e2], p2);
+                  // 255 P~ + 1.5 * 2^23: one rounding to the nearest integer (ties to even); the
+                  // integer sits in the low byte of the result (P~ <= 1).
+                  const float2 y2 = __ffma2_rn(p2, c255, magic2);
+                  y[2 * e2] = __float_as_uint(y2.x);
+                  y[2 * e2 + 1] = __float_as_uint(y2.y);
+                  if (CHECK) {
+                    // Distance of 255 P~ from the code it rounded to; near 1/2 the fast
+                    // exponential's error can decide the code.
+                    const float2 r2 = __ffma2_rn(p2, c255, __fadd2_rn(magic2, make_float2(-y2.x, -y2.y)));
+                    rmx = fmax3(rmx, fabsf(r2.x), fabsf(r2.y));
+                  }
+                }
+                pk[w] = __byte_perm(__byte_perm(y[0], y[1], 0x0040), __byte_perm(y[2], y[3], 0x0040), 0x5410);
+              }
+              if (CHECK && rmx > kTieBand) {
+                // Rare: settle this group's near-tie codes one key at a time (a rolled loop over a
+                // small local copy, so the double-precision exponential appears once).
+                float sg[16];
+                uint32_t pw[4];
+#pragma unroll
+                for (int k = 0; k < 16; ++k) sg[k] = __uint_as_float(x[16 * g4 + k]);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) pw[k] = pk[4 * g4 + k];
+#pragma unroll 1
+                for (int k = 0; k < 16; ++k) {
+                  const float pk1 = ex2_approx(__fmul_rn(__fadd_rn(sg[k], -m_new), kLog2e));
+                  const float rk = __fmaf_rn(pk1, 255.0f, __fadd_rn(kMagic, -__fmaf_rn(pk1, 255.0f, kMagic)));
+                  if (fabsf(rk) > kTieBand) {
+                    const uint32_t code = exact_code(sg[k], m_new);
+                    const uint32_t sh = 8u * static_cast<uint32_t>(k & 3);
+                    pw[k >> 2] = (pw[k >> 2] & ~(0xFFu << sh)) | (code << sh);
+                  }
+                }
+#pragma unroll
+                for (int k = 0; k < 4; ++k) pk[4 * g4 + k] = pw[k];
+              }
+            }
+            tmem_st_cols<8>(aS + 8 * c, pk);
+            if (p.dbg_p != nullptr && row_ok) {
+#pragma unroll
+              for (int k = 0; k < 32; ++k)
+                if (32 * c + k < nk)
+                  p.dbg_p[(bh * N + i) * N + j0 + 32 * c + k] = static_cast<uint8_t>(pk[k >> 2] >> (8 * (k & 3)));
             }
           }
-          if (ok && t > 0) tc_commit(&bars[Bar::kvempty((t - 1) % S)]);
+        };
+        if (check)
+          pass2(std::true_type{});
+        else
+          pass2(std::false_type{});
+        const float lt = (lt2[0].x + lt2[0].y) + (lt2[1].x + lt2[1].y);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[Bar::pfull(grp)]);
+
+        // ---- fold block n: F' += acc e_n, L' += l_n e_n (after P.V(n), which followed the fold
+        // of block n - 1; at an item's first block also after both groups' previous epilogue)
+        if (!wait_warp(&bars[Bar::pvdone(grp)], (n >> 1) & 1, abort_flag)) {
+          alive = false;
+          break;
         }
+        if (n > 0 && !wait_warp(&bars[Bar::folddone(grp ^ 1)], ((n - 1) >> 1) & 1, abort_flag)) {
+          alive = false;
+          break;
+        }
+        if (t == 0 && it > 0 && !wait_warp(&bars[Bar::epidone()], (it - 1) & 1, abort_flag)) {
+          alive = false;
+          break;
+        }
+        tc_fence_after();
+        {
+          float e = 1.0f, ratio = 1.0f;
+          float mref = m_new, Lp = 0.0f;
+          if (t > 0) {
+            const float2 lm = s_Lm[r];
+            Lp = lm.x;
+            mref = lm.y;
+            e = ex2_approx((m_new - mref) * kLog2e);
+            if (e > 1.8446744e19f) {  // 2^64: move the reference up to m_n, rescaling F' and L'
+              ratio = 1.0f / e;
+              e = 1.0f;
+              mref = m_new;
+            }
+          }
+          const bool rescale = __any_sync(0xffffffffu, ratio != 1.0f);
+          auto fold = [&](auto first) {
+            constexpr bool FIRST = decltype(first)::value;  // the item's first block: F' = acc
+#pragma unroll 1
+            for (int c0 = 0; c0 < DP; c0 += 32) {
+              constexpr int G = 32;
+              uint32_t a[G], f[G];
+              if (c0 + G <= DP) {
+                tmem_ld_cols<G>(aAcc + c0, a);
+                if (!FIRST) tmem_ld_cols<G>(aF + c0, f);
+              } else {
+                tmem_ld_cols<16>(aAcc + c0, a);
+                if (!FIRST) tmem_ld_cols<16>(aF + c0, f);
+              }
+              tmem_ld_wait();
+              reg_fence_cols<G>(a);
+              if (!FIRST) reg_fence_cols<G>(f);
+              const float2 e2 = make_float2(e, e), rt2 = make_float2(ratio, ratio);
+#pragma unroll
+              for (int k = 0; k < G; k += 2) {
+                const float2 a2 = __fadd2_rn(
+                    make_float2(__uint_as_float(a[k] + kMagicBits), __uint_as_float(a[k + 1] + kMagicBits)),
+                    make_float2(-kMagic, -kMagic));
+                float2 f2;
+                if (FIRST) {
+                  f2 = a2;
+                } else {
+                  float2 fo = make_float2(__uint_as_float(f[k]), __uint_as_float(f[k + 1]));
+                  if (rescale) fo = __fmul2_rn(fo, rt2);
+                  f2 = __ffma2_rn(a2, e2, fo);
+                }
+                f[k] = __float_as_uint(f2.x);
+                f[k + 1] = __float_as_uint(f2.y);
+              }
+              if (c0 + G <= DP)
+                tmem_st_cols<G>(aF + c0, f);
+              else
+                tmem_st_cols<16>(aF + c0, f);
+            }
+          };
+          if (t == 0)
+            fold(std::true_type{});
+          else
+            fold(std::false_type{});
+          own_L = (t == 0) ? lt : __fmaf_rn(lt, e, Lp * ratio);
+          own_mref = mref;
+          s_Lm[r] = make_float2(own_L, own_mref);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[Bar::folddone(grp)]);
       }
-      // Every MMA this thread issued has completed before tensor memory is released.
-      tc_commit(&bars[Bar::drain()]);
-      wait_bounded(&bars[Bar::drain()], 0, abort_flag, false);
-    }
-    __syncwarp();
-  } else if (warp >= 4) {
-    // ------------------------------------------------------------ softmax warpgroups
-    const int q = (warp - 4) >> 2, w4 = warp & 3;
-    const int r = w4 * 32 + lane;
-    const int i = q0 + q * BM + r;
-    const bool row_ok = i < N;
-    const int ic = row_ok ? i : N - 1;  // rows past N read the bias of row N-1 (never stored)
-    const uint32_t lane_base = static_cast<uint32_t>(w4 * 32) << 16;
-    const uint32_t aS = tmem + lane_base + C::tS(q);
-    const uint32_t aP = tmem + lane_base + C::tP(q);
-    const uint32_t aO0 = tmem + lane_base + C::tO(q, 0);
-    const uint32_t aO1 = tmem + lane_base + C::tO(q, 1);
-    const uint32_t aF = tmem + lane_base + C::tF(q);  // unused when F is in shared memory
-    const float alpha = __fmul_rn(__fmul_rn(p.softmax_scale, p.mu_q[bh]), p.mu_k[bh]);
-    const float2 alpha2 = make_float2(alpha, alpha);
+      if (!alive) break;
 
-    // Bias addressing. Dense: this row of [H][N][N]. Rel-pos: b_ij = tab[a_i - koff_j] with
-    // tab the head's table (staged in shared memory when it fits, followed by zeros that
-    // class-token rows and keys index into), koff_j kept as byte offsets.
-    const float* brow = nullptr;
-    const float* gtab = nullptr;
-    int a_i = 0;
-    if (BK == BA_BIAS_DENSE) brow = p.bias.data + b * p.bias.batch_stride + (h * N + ic) * N;
-    if (is_relpos(BK)) {
-      const int W2 = 2 * p.bias.table_w - 1;
-      gtab = p.bias.data + h * static_cast<int64_t>(2 * p.bias.table_h - 1) * W2;
-      if (ic >= p.bias.n_prefix) {
-        const int ti = ic - p.bias.n_prefix;
-        const int yi = ti / p.bias.grid_w;
-        a_i = (yi + p.bias.table_h - 1) * W2 + (ti - yi * p.bias.grid_w) + p.bias.table_w - 1;
-      } else {
-        a_i = (tab_mode == 2) ? tsize + kmax : -1;  // class-token row: the zeros (or the general path)
+      // ---- epilogue: O = F' v_scale / (255 L'), channels 64 grp .. (DP / 2 per group), once
+      // the item's last block is folded; then both groups release F' for the next item.
+      if (it + 1 < n_items) {
+        int64_t nbh;
+        int nq0;
+        item_at(by_head, it + 1, p.H, nqb, BM, nbh, nq0);
+        mu_q_next = p.mu_q[nbh];
+        mu_k_next = p.mu_k[nbh];
       }
-    }
-    const uint32_t tb = smem_u32(stab) + 4u * static_cast<uint32_t>(a_i);  // this row's table base
-    // Fast path: full key blocks, no debug output, aligned dense rows, rel-pos table in shared
-    // memory with the class tokens handled by the zero padding.
-    const bool fast_ok = (p.dbg_logits == nullptr) &&
-                         (BK != BA_BIAS_DENSE || ((N & 3) == 0 && (p.bias.batch_stride & 3) == 0)) &&
-                         (!is_relpos(BK) || p.bias.n_prefix == 0 || tab_mode == 2);
-    const float* grow = gtab + a_i;  // this row's base in a table left in global memory
-
-    float m = -CUDART_INF_F, l = 0.0f;
-    bool alive = true;
-    // Accumulator that P.V of the current block adds into (tile-uniform), whether F holds
-    // anything yet, and how many blocks that accumulator holds.
-    int cur = 0, nblk = 1;
-    bool f_valid = false;
-
-    for (int t = 0; t < T && alive; ++t) {
-      const int st = t % S;
-      const int nk = min(BN, N - t * BN);
-      // 32-key chunks that hold keys of this block. The P codes of the chunks past them are
-      // left as they are: they multiply V rows past N, which the V copy fills with zeros.
-      const int nch = (nk + 31) >> 5;
-      if (is_relpos(BK) && !wait_warp(&bars[Bar::kvfull(st)], (t / S) & 1, abort_flag)) {
-        alive = false;
-        break;
-      }
-      if (!wait_warp(&bars[Bar::sfull(q)], t & 1, abort_flag)) {
+      const int nl = n0 + T - 1;  // the item's last block
+      if (!wait_warp(&bars[Bar::folddone(nl & 1)], (nl >> 1) & 1, abort_flag)) {
         alive = false;
         break;
       }
       tc_fence_after();
-      const uint32_t ko_s = smem_u32(koff + st * BN);
-
-      // Pass 1: s = alpha * x + b written back over S in TMEM; block max. The next 32-column
-      // block is loaded from TMEM while this one is computed.
-      float mx[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
-      // The fast path also takes a partial last block (keys past N are masked to -inf after
-      // the fact; their rel-pos offsets point at valid entries), except for dense bias rows,
-      // which end at N.
-      const bool fast = fast_ok && (nk == BN || BK != BA_BIAS_DENSE);
-      {
-        // One copy of the block body (a small hot loop stays in the instruction cache; the
-        // other softmax warps of the SM cover the TMEM load latency).
-#pragma unroll 1
-        for (int c = 0; c < nch; ++c) {
-          uint32_t x[32];
-          tmem_ld32(aS + 32 * c, x);
-          tmem_ld_wait();
-          reg_fence32(x);
-          if (fast) {
-            if (nk == BN)
-              fast_block<BK, false>(x, c, nk, alpha2, brow + t * BN, ko_s, tb, grow, tab_mode, mx);
-            else
-              fast_block<BK, true>(x, c, nk, alpha2, brow + t * BN, ko_s, tb, grow, tab_mode, mx);
-          } else {
-            // General path: a partial last block, class tokens without zero padding,
-            // unaligned dense rows, a table in global memory, or the debug logits.
-#pragma unroll
-            for (int u = 0; u < 32; ++u) {
-              const int j = 32 * c + u;
-              float sv = -CUDART_INF_F;
-              if (j < nk) {
-                const float xf = __uint_as_float(x[u]);
-                float bias = 0.0f;
-                if (BK == BA_BIAS_DENSE) bias = __ldg(brow + t * BN + j);
-                if (is_relpos(BK)) {
-                  const int kj = lds_s32(ko_s + 4u * j) >> 2;
-                  if (a_i >= 0 && kj >= 0)
-                    bias = (tab_mode != 0) ? lds_f32(smem_u32(stab) + 4u * static_cast<uint32_t>(a_i - kj))
-                                           : __ldg(gtab + (a_i - kj));
-                }
-                sv = __fmaf_rn(alpha, xf, bias);
-                if (p.dbg_logits != nullptr && row_ok)
-                  p.dbg_logits[(bh * N + i) * N + t * BN + j] = __float2int_rn(xf);
-              }
-              mx[u & 3] = fmaxf(mx[u & 3], sv);
-              x[u] = __float_as_uint(sv);
-            }
-          }
-          tmem_st32(aS + 32 * c, x);
-        }
-      }
-      const float m_new = fmaxf(m, fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])));
-      tmem_st_wait();
-
-      // Pass 2: P~ = 2^((s - m) log2 e) (masked keys hold s = -inf: P~ = 0), row sum, u8 codes
-      // -> TMEM columns 0..31 (their s values were read in the first step of this pass).
-      const float2 negm2 = make_float2(-m_new, -m_new);
-      const float2 log2e2 = make_float2(kLog2e, kLog2e);
-      const float2 c255 = make_float2(255.0f, 255.0f);
-      const float2 magic2 = make_float2(12582912.0f, 12582912.0f);
-      float2 lt2[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
-      {
-#pragma unroll 1
-        for (int c = 0; c < nch; ++c) {
-          uint32_t x[32];
-          tmem_ld32(aS + 32 * c, x);
-          tmem_ld_wait();
-          reg_fence32(x);
-          uint32_t pk[8];
-#pragma unroll
-          for (int w = 0; w < 8; ++w) {
-            uint32_t y[4];
-#pragma unroll
-            for (int e2 = 0; e2 < 2; ++e2) {
-              const int u = 4 * w + 2 * e2;
-              // s - m first (exact near the max), then the scale to base 2.
-              const float2 t2 = __fmul2_rn(
-                  __fadd2_rn(make_float2(__uint_as_float(x[u]), __uint_as_float(x[u + 1])), negm2), log2e2);
-              const float2 p2 = ((kPolyPairs >> (2 * w + e2)) & 1u) ? exp2_poly2(t2)
-                                                                    : make_float2(ex2_approx(t2.x), ex2_approx(t2.y));
-              lt2[e2] = __fadd2_rn(lt2[e2], p2);
-              // 255 P~ + 1.5 * 2^23: one rounding to the nearest integer (ties to even); the
-              // integer sits in the low byte of the result (P~ <= 1).
-              const float2 y2 = __ffma2_rn(p2, c255, magic2);
-              y[2 * e2] = __float_as_uint(y2.x);
-              y[2 * e2 + 1] = __float_as_uint(y2.y);
-            }
-            pk[w] = __byte_perm(__byte_perm(y[0], y[1], 0x0040), __byte_perm(y[2], y[3], 0x0040), 0x5410);
-          }
-          tmem_st8(aP + 8 * c, pk);
-        }
-      }
-      const float lt = (lt2[0].x + lt2[0].y) + (lt2[1].x + lt2[1].y);
-      // Rescale factor of the row's earlier blocks: exactly 1 while its max is unchanged.
-      const float ct = (m == -CUDART_INF_F) ? 0.0f : (m_new > m ? ex2_approx((m - m_new) * kLog2e) : 1.0f);
-      l = l * ct + lt;
-      // Vote (per warp) whether a row raised its max; the MMA thread reads the votes of the
-      // tile's four warps after their p_full arrivals.
-      const bool rose = __any_sync(0xffffffffu, t > 0 && m_new > m);
-      if (lane == 0) votes[((t & 1) * NQ + q) * 4 + w4] = rose ? 1u : 0u;
-      m = m_new;
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[Bar::pfull(q)]);
-      if (t == 0) continue;
-      // While the MMAs of the next block run: if any row of the tile raised its max, P.V of
-      // this block goes to the other accumulator, and the old one is folded into F with this
-      // row's factor (1 for rows whose max did not rise).
-      if (!wait_warp(&bars[Bar::pfull(q)], t & 1, abort_flag)) {
-        alive = false;
-        break;
-      }
-      const volatile uint32_t* vt = votes + ((t & 1) * NQ + q) * 4;
-      if ((vt[0] | vt[1] | vt[2] | vt[3]) != 0u) {
-        fold_rest<C, 0>(cur ? aO1 : aO0, aF, sF + q * BM + r, make_float2(ct, ct), !f_valid, nblk == 1);
-        if (!C::kFSmem) tmem_st_wait();
-        cur ^= 1;
-        f_valid = true;
-        nblk = 1;
-      } else {
-        ++nblk;
-      }
-    }
-
-    if (alive && wait_warp(&bars[Bar::odone(q)], 0, abort_flag)) {
-      tc_fence_after();
-      const float inv_l = 1.0f / l;
-      // Rows whose byte length is a multiple of 16 are written with 16-byte stores (each
-      // thread owns one row); other shapes fall back to element stores.
+      const float inv_l = 1.0f / (255.0f * s_Lm[r].x);
       const int esz = (p.o_dt == BA_F32) ? 4 : 2;
       const bool vec = ((d * esz) & 15) == 0;
-      char* orow = reinterpret_cast<char*>(p.o) + ((bh * N + i) * d) * esz;
-      const uint32_t aO = cur ? aO1 : aO0;
-      const float4* fr = sF + q * BM + r;
 #pragma unroll 1
-      for (int cc = 0; cc < DP / 16; ++cc) {
-        uint32_t a[16];
-        float f[16];
-        tmem_ld16(aO + 16 * cc, a);
-        if constexpr (C::kFSmem) {
-          tmem_ld_wait();
-          reg_fence16(a);
+      for (int g0 = 0; g0 < DH; g0 += 8) {
+        const int c0 = grp * DH + g0;  // eight channels at a time of this group's DH
+        uint32_t f[8];
+        tmem_ld_cols<8>(aF + c0, f);
+        tmem_ld_wait();
+        reg_fence8(f);
+        float val[8];
 #pragma unroll
-          for (int k4 = 0; k4 < 4; ++k4) {
-            const float4 v = f_valid ? fr[(4 * cc + k4) * (NQ * BM)] : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-            f[4 * k4] = v.x; f[4 * k4 + 1] = v.y; f[4 * k4 + 2] = v.z; f[4 * k4 + 3] = v.w;
-          }
-        } else {
-          uint32_t fb[16];
-          if (f_valid) tmem_ld16(aF + 16 * cc, fb);
-          tmem_ld_wait();
-          reg_fence16(a);
-          if (f_valid) reg_fence16(fb);
-#pragma unroll
-          for (int e = 0; e < 16; ++e) f[e] = f_valid ? __uint_as_float(fb[e]) : 0.0f;
+        for (int k = 0; k < 8; ++k) {
+          const float sv = (c0 + k < d) ? __ldg(p.v_scale + bh * d + c0 + k) : 0.0f;
+          val[k] = __uint_as_float(f[k]) * (sv * inv_l);
         }
-        float val[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e)
-          val[e] = (f[e] + __int2float_rn(static_cast<int>(a[e]))) * sscale[16 * cc + e] * inv_l;
         if (!row_ok) continue;
-        if (vec && 16 * cc + 16 <= d) {
+        char* orow = reinterpret_cast<char*>(p.o) + ((bh * N + i) * d + c0) * esz;
+        if (vec && c0 + 8 <= d) {
           if (p.o_dt == BA_F32) {
-#pragma unroll
-            for (int k4 = 0; k4 < 4; ++k4)
-              reinterpret_cast<float4*>(orow + (16 * cc + 4 * k4) * 4)[0] =
-                  make_float4(val[4 * k4], val[4 * k4 + 1], val[4 * k4 + 2], val[4 * k4 + 3]);
+            reinterpret_cast<float4*>(orow)[0] = make_float4(val[0], val[1], val[2], val[3]);
+            reinterpret_cast<float4*>(orow)[1] = make_float4(val[4], val[5], val[6], val[7]);
           } else {
-            uint32_t h[8];
+            uint32_t hw[4];
 #pragma unroll
-            for (int k2 = 0; k2 < 8; ++k2) {
+            for (int k2 = 0; k2 < 4; ++k2) {
               if (p.o_dt == BA_F16) {
-                const __half2 v = __floats2half2_rn(val[2 * k2], val[2 * k2 + 1]);
-                h[k2] = *reinterpret_cast<const uint32_t*>(&v);
+                const __half2 hv = __floats2half2_rn(val[2 * k2], val[2 * k2 + 1]);
+                hw[k2] = *reinterpret_cast<const uint32_t*>(&hv);
               } else {
-                const __nv_bfloat162 v = __floats2bfloat162_rn(val[2 * k2], val[2 * k2 + 1]);
-                h[k2] = *reinterpret_cast<const uint32_t*>(&v);
+                const __nv_bfloat162 hv = __floats2bfloat162_rn(val[2 * k2], val[2 * k2 + 1]);
+                hw[k2] = *reinterpret_cast<const uint32_t*>(&hv);
               }
             }
-            reinterpret_cast<uint4*>(orow + 16 * cc * 2)[0] = make_uint4(h[0], h[1], h[2], h[3]);
-            reinterpret_cast<uint4*>(orow + 16 * cc * 2)[1] = make_uint4(h[4], h[5], h[6], h[7]);
+            reinterpret_cast<uint4*>(orow)[0] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
           }
         } else {
 #pragma unroll
-          for (int e = 0; e < 16; ++e)
-            if (16 * cc + e < d) store_out(p.o, (bh * N + i) * d + 16 * cc + e, val[e], p.o_dt);
+          for (int k = 0; k < 8; ++k)
+            if (c0 + k < d) store_out(p.o, (bh * N + i) * d + c0 + k, val[k], p.o_dt);
         }
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[Bar::epidone()]);
     }
   }
 
@@ -1437,7 +1035,7 @@ __global__ void __launch_bounds__(Cfg<DP, NQ_>::kThreads, Cfg<DP, NQ_>::kCtasPer
   named_barrier_sync(1, C::kThreads);
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, C::kTmemCols);
+    tmem_dealloc(tmem, 512);
   }
 }
 
@@ -1458,53 +1056,49 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-constexpr int kMaxSmem = 227 * 1024;      // per CTA
-constexpr int kSmPerSmem = 228 * 1024;    // per SM
-constexpr int kSmemReserved = 1024;       // per CTA, taken by the runtime
-
-// Dynamic shared memory a CTA of configuration C may use.
-template <class C>
-constexpr int smem_room() {
-  return C::kCtasPerSm == 1 ? kMaxSmem : kSmPerSmem / C::kCtasPerSm - kSmemReserved;
-}
+constexpr int kMaxSmem = 227 * 1024;  // per CTA
 
 // 0: rel-pos table read from global memory; 1: staged in shared memory; 2: staged and followed
 // by 2 * tsize zeros that class-token rows and keys index into.
 template <class C>
 int relpos_table_mode(const AttnParams& p) {
   const int64_t tsize = static_cast<int64_t>(2 * p.bias.table_h - 1) * (2 * p.bias.table_w - 1);
-  const int64_t room = smem_room<C>() - 1024 - C::kTabOff;
+  const int64_t room = kMaxSmem - 1024 - C::kTabOff;
   if (p.bias.n_prefix > 0 && 3 * tsize * 4 <= room) return 2;
   if (tsize * 4 <= room) return 1;
   return 0;
 }
 
-template <int DP, int BK, int NQ>
-constexpr auto pick_kernel() {
-  if constexpr (DP > 80)
-    return attn_tc_single_kernel<DP, BK, NQ>;
-  else
-    return attn_tc_kernel<DP, BK, NQ>;
+// Row stride of the rel-pos window, or 0 when the window form does not apply: it needs a grid
+// width that is a multiple of 32 (so that every 32-key chunk lies in one grid row), no class
+// tokens, and a window of at most kWinFloats entries for every (tile, block) pair. A run of 128
+// tokens spans at most 127 / gw + 2 grid rows; the dx extent is at most 255 when the tiles and
+// blocks cannot straddle grid rows (gw a multiple of 128), else 2 gw - 1.
+int window_stride(const AttnParams& p) {
+  if (p.bias.kind != BA_BIAS_RELPOS2D || p.bias.n_prefix != 0) return 0;
+  const int gw = p.bias.grid_w;
+  if (gw % 32 != 0) return 0;
+  const int ws = (gw % 128 == 0) ? 256 : ((2 * gw - 1 + 3) / 4) * 4;
+  const int ndy = 2 * (127 / gw + 2) - 1;
+  return static_cast<int64_t>(ndy) * ws <= kWinFloats ? ws : 0;
 }
 
-template <int DP, int BK, int NQ>
+template <int DP, int BK>
 cudaError_t launch_cfg(const AttnParams& p, const CUtensorMap& tm, cudaStream_t s) {
-  using C = Cfg<DP, NQ>;
-  int tab_mode = 0, tsize = 0, kmax = 0;
-  if (is_relpos(BK)) {
+  using C = Cfg<DP, BK>;
+  int tab_mode = 0, tsize = 0, kmax = 0, wst = 0;
+  if (BK == kRelSmem || BK == kRelGlobal || BK == kRelWindow) {
     tsize = (2 * p.bias.table_h - 1) * (2 * p.bias.table_w - 1);
     kmax = (p.bias.grid_h - 1) * (2 * p.bias.table_w - 1) + p.bias.grid_w - 1;
-    tab_mode = relpos_table_mode<C>(p);
   }
+  if (BK == kRelSmem) tab_mode = relpos_table_mode<C>(p);
+  if (BK == kRelWindow) wst = window_stride(p);
   const int tab_bytes = tab_mode == 0 ? 0 : (tab_mode == 2 ? 3 : 1) * tsize * 4;
-  // A CTA that owns all 512 tensor-memory columns takes enough shared memory to be alone on its
-  // SM; one that owns 256 takes enough that no third CTA fits.
+  // One CTA per SM (it owns all 512 tensor-memory columns): take enough shared memory that no
+  // second CTA is placed beside it.
   int smem = C::kTabOff + tab_bytes + 1024;
-  const int floor_bytes = C::kCtasPerSm == 1 ? 116 * 1024 : 80 * 1024;
-  if (smem < floor_bytes) smem = floor_bytes;
-  // Heads wider than 80 channels: one work item per CTA; otherwise the persistent kernel.
-  constexpr bool kSingle = DP > 80;
-  auto kernel = pick_kernel<DP, BK, NQ>();
+  if (smem < 116 * 1024) smem = 116 * 1024;
+  auto kernel = attn_tc_kernel<DP, BK>;
   static int configured = 0;
   if (smem > configured) {
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -1513,66 +1107,45 @@ cudaError_t launch_cfg(const AttnParams& p, const CUtensorMap& tm, cudaStream_t 
     if (e != cudaSuccess) return e;
     configured = smem;
   }
-  // Persistent CTAs: as many as fit at once (CTAs per SM x SMs), H per group, each walking the
-  // items of its head; at least one CTA per head.
   int dev = 0, sms = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
+  // Persistent CTAs, one per SM; grouped by head (at least one CTA per head) when the head's
+  // table is staged.
   const int64_t per_head = static_cast<int64_t>(p.B) * ceil_div(p.N, BM * C::NQ);
-  const int64_t slots = static_cast<int64_t>(C::kCtasPerSm) * sms;
   int64_t grid;
-  if (kSingle) {
-    grid = per_head * p.H;
-  } else if (is_relpos(BK) && tab_mode != 0) {  // items grouped by head (the kernel's by_head)
-    const int64_t k = std::max<int64_t>(1, std::min<int64_t>(per_head, slots / p.H));
+  if (BK == kRelSmem) {
+    const int64_t k = std::max<int64_t>(1, std::min<int64_t>(per_head, sms / p.H));
     grid = k * p.H;
   } else {
-    grid = std::min<int64_t>(per_head * p.H, slots);
+    grid = std::min<int64_t>(per_head * p.H, sms);
   }
-  if constexpr (kSingle) {
-    kernel<<<static_cast<unsigned>(grid), C::kThreads, smem, s>>>(p, tm, tab_mode, tsize, kmax);
-    return cudaGetLastError();
-  } else {
-    // Programmatic dependent of the preparation kernel: the launch, and the barrier set-up of
-    // the CTAs that find an SM free, overlap the last preparation CTAs; each CTA waits for the
-    // preparation grid (grid_dependency_wait) before it reads anything that grid writes.
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(grid));
-    cfg.blockDim = dim3(C::kThreads);
-    cfg.dynamicSmemBytes = static_cast<size_t>(smem);
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kernel, p, tm, tab_mode, tsize, kmax);
-  }
+  // Programmatic dependent of the preparation kernel: the launch, and the barrier set-up of
+  // the CTAs that find an SM free, overlap the last preparation CTAs; each CTA waits for the
+  // preparation grid (grid_dependency_wait) before it reads anything that grid writes.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(C::kThreads);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, p, tm, tab_mode, tsize, kmax, wst);
 }
 
-template <int DP, int NQ>
-cudaError_t launch_nq(const AttnParams& p, const CUtensorMap& tm, cudaStream_t s) {
-  switch (p.bias.kind) {
-    case BA_BIAS_DENSE: return launch_cfg<DP, BA_BIAS_DENSE, NQ>(p, tm, s);
-    case BA_BIAS_RELPOS2D:
-      return relpos_table_mode<Cfg<DP, NQ>>(p) != 0 ? launch_cfg<DP, BA_BIAS_RELPOS2D, NQ>(p, tm, s)
-                                                     : launch_cfg<DP, kRelposGlobal, NQ>(p, tm, s);
-    default: return launch_cfg<DP, BA_BIAS_NONE, NQ>(p, tm, s);
-  }
-}
-
-// Head dimensions up to 64 run one query tile per CTA in half of tensor memory, two CTAs per
-// SM (the CTAs' prologues, pipeline fills and epilogues overlap each other's work), unless the
-// rel-pos table only fits in the shared memory of a CTA that has the SM to itself; then one CTA
-// runs two tiles.
 template <int DP>
 cudaError_t launch_dp(const AttnParams& p, const CUtensorMap& tm, cudaStream_t s) {
-  if constexpr (DP <= 64) {
-    const bool table_fits = p.bias.kind != BA_BIAS_RELPOS2D || relpos_table_mode<Cfg<DP, 1>>(p) != 0;
-    return table_fits ? launch_nq<DP, 1>(p, tm, s) : launch_nq<DP, 2>(p, tm, s);
-  } else {
-    return launch_nq<DP, 1>(p, tm, s);
+  switch (p.bias.kind) {
+    case BA_BIAS_DENSE: return launch_cfg<DP, kBiasDense>(p, tm, s);
+    case BA_BIAS_RELPOS2D:
+      if (window_stride(p) != 0) return launch_cfg<DP, kRelWindow>(p, tm, s);
+      return relpos_table_mode<Cfg<DP, kRelSmem>>(p) != 0 ? launch_cfg<DP, kRelSmem>(p, tm, s)
+                                                          : launch_cfg<DP, kRelGlobal>(p, tm, s);
+    default: return launch_cfg<DP, kBiasNone>(p, tm, s);
   }
 }
 
@@ -1598,6 +1171,11 @@ cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t s) {
                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                          CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+#ifdef BA_TEST_SKIP_ARRIVE
+  // Test build: one kernel variant (d = 64, no bias) is enough to exercise the bounded waits.
+  if (p.dp != 64 || p.bias.kind != BA_BIAS_NONE) return cudaErrorNotSupported;
+  return launch_cfg<64, kBiasNone>(p, tm, s);
+#endif
   switch (p.dp) {
     case 16: return launch_dp<16>(p, tm, s);
     case 32: return launch_dp<32>(p, tm, s);

@@ -117,6 +117,8 @@ struct AttnParams {
   void* o;
   int o_dt;
   int32_t* dbg_logits;
+  uint8_t* dbg_p;   // debug: the 8-bit codes P_ij [B][H][N][N], or null
+  int p_check_all;  // recompute every near-tie code exactly, not only where it could matter
 };
 
 }  // namespace binattn

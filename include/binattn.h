@@ -148,6 +148,25 @@ ba_status ba_attention_fwd(const void* q, const void* k, const void* v, ba_dtype
                            void* stream);
 
 /*
+ * ba_attention_fwd with debug outputs, for tests and diagnosis (slower; not for production use).
+ *   dbg_logits:      NULL, or [B][H][N][N] int32 receiving x_ij.
+ *   dbg_p:           NULL, or [B][H][N][N] uint8 receiving the 8-bit code P_ij of every key, taken
+ *                    against the running maximum of the key's block (the codes the P.V product
+ *                    uses; gist.science/zh 2.2(3)).
+ *   check_all_codes: 0 = as ba_attention_fwd: the tensor-core kernel evaluates exp with the
+ *                    hardware approximation and recomputes from the double-precision exponential
+ *                    every code within its error band of a rounding tie in those blocks where a
+ *                    changed code could move the output by more than a tenth of the 2e-3 error
+ *                    bar (rows whose softmax sum is still small); 1 = in every block, so that every
+ *                    code equals the definition's.  Other values: BA_ERR_INVALID_ARG.
+ *   Other arguments and errors as ba_attention_fwd (dbg_p must be 16-byte aligned).
+ */
+ba_status ba_attention_fwd_debug(const void* q, const void* k, const void* v, ba_dtype dt, int B, int H,
+                                 int N, int d, const ba_bias* bias, float softmax_scale, void* o,
+                                 ba_dtype o_dt, void* ws, size_t ws_bytes, int32_t* dbg_logits,
+                                 uint8_t* dbg_p, int check_all_codes, void* stream);
+
+/*
  * ba_attention_fwd without a caller-supplied workspace (the paper has no counterpart; this
  * is a deployment convenience). For callers that cannot allocate device memory: a plugin that
  * is handed only its input and output buffers, or a runtime that fixes all device memory at

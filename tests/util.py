@@ -35,6 +35,12 @@ def oracle_forward(w, rows=None, num_threads=0, softmax_scale=0.0):
                                       num_threads=num_threads, rows=rows)
 
 
+def oracle_forward_debug(w, rows=None):
+    """The oracle's O and its per-row diagnostics (8-bit codes "pu8" [rows, N], ...)."""
+    q, k, v = oracle_qkv(w)
+    return oracle.get().attention_fwd(q, k, v, oracle_bias(w), block_c=128, rows=rows, debug=True)
+
+
 def sample_rows(N: int, n: int = 48, seed: int = 0) -> np.ndarray:
     """First and last rows (the ragged tail) plus random rows in between, sorted."""
     rng = np.random.default_rng(seed)
