@@ -329,9 +329,14 @@ def main():
         prep_bytes = {"stream_qkv": 3 * E * esz + 2 * BH * N * 16 + BH * N * dp + BH * 4 * (d + 2),
                       "finalize": 0, "quant_v": 0}
     else:
-        prep_bytes = {"stream_qkv": 3 * E * esz + 2 * BH * N * 16 + BH * nchunk * (8 + 4 * dp),
-                      "finalize": BH * nchunk * (8 + 4 * dp) + BH * (8 + 8 * dp),
-                      "quant_v": E * esz + BH * N * dp + BH * 4 * dp}
+        # two launches: the streaming kernel reads q, k, v and writes sign rows, per-chunk |x| sums
+        # and per-group V channel maxima; the quantiser reads V again (the scales need the whole
+        # slice's maxima first) and the partials, and writes int8 V, the scales and mu
+        nparts = -(-nchunk // 8) if d % 8 == 0 else nchunk
+        partials = 2 * BH * nchunk * 8 + BH * nparts * dp * 4
+        prep_bytes = {"stream_qkv": 3 * E * esz + 2 * BH * N * 16 + partials,
+                      "finalize": 0,
+                      "quant_v": E * esz + partials + BH * N * dp + BH * 4 * (d + 2)}
     alg_bytes = {
         **prep_bytes,
         "attention": 2 * BH * N * 16 + BH * N * dp + E * esz + bias_bytes + BH * 4 * (d + 2),
@@ -410,8 +415,8 @@ def main():
             "roofline": roof,
             "cpu_baseline": cpu,
             "e2e": e2e,
-            # prep (1 launch on the one-launch path, else prep + finalize + quantise) + attention
-            "gpu_launches": ((2 if ba.prep_fused(w.B, w.H, w.N, w.d) else 4) * args.steps),
+            # prep (1 launch on the one-launch path, else streaming + quantiser) + attention
+            "gpu_launches": ((2 if ba.prep_fused(w.B, w.H, w.N, w.d) else 3) * args.steps),
             "clocks": clk,
         }
         print(json.dumps(line), flush=True)

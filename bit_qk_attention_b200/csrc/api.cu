@@ -95,7 +95,7 @@ PrepDims dims(int B, int H, int N, int d) {
 // Workspace regions (byte offsets, each 256-byte aligned).
 struct WsLayout {
   size_t bits_q = 0, bits_k = 0, mu_q = 0, mu_k = 0, vq = 0, v_scale = 0;
-  size_t part_mu_q = 0, part_mu_k = 0, part_amax = 0, inv = 0, total = 0;
+  size_t part_mu_q = 0, part_mu_k = 0, part_amax = 0, total = 0;
 };
 
 enum { kWsPack = 1, kWsQuant = 2, kWsAll = 3 };
@@ -123,8 +123,7 @@ WsLayout layout(int B, int H, int N, int d, int what) {
     if (what == kWsAll) L.part_mu_k = take(static_cast<size_t>(g.BH) * g.nchunk * 8);
   }
   if (what & kWsQuant) {
-    L.part_amax = take(static_cast<size_t>(g.BH) * g.nchunk * g.dp * 4);
-    L.inv = take(static_cast<size_t>(g.BH) * g.dp * 4);
+    L.part_amax = take(static_cast<size_t>(g.BH) * amax_parts(g) * g.dp * 4);
   }
   L.total = off;
   return L;
@@ -278,18 +277,14 @@ ba_status ba_quant_v(const void* v, ba_dtype dt, int B, int H, int N, int d, int
   pp.job[0] = PrepJob{v, kJobAmax, nullptr, nullptr, at<float>(ws, L.part_amax)};
   pp.job[1] = pp.job[2] = pp.job[0];
   if ((st = cuda_status(launch_prep(pp, dt, 1, s))) != BA_OK) return st;
-  FinalizeParams fp{};
-  fp.g = g;
-  fp.npack = 0;
-  fp.part_amax = at<float>(ws, L.part_amax);
-  fp.inv = at<float>(ws, L.inv);
-  fp.v_scale = v_scale;
-  if ((st = cuda_status(launch_finalize(fp, s))) != BA_OK) return st;
   QuantParams qp{};
   qp.g = g;
   qp.v = v;
-  qp.inv = at<float>(ws, L.inv);
+  qp.part_amax = at<float>(ws, L.part_amax);
+  qp.npart = amax_parts(g);
+  qp.v_scale = v_scale;
   qp.vq = vq;
+  qp.npack = 0;
   return cuda_status(launch_quant(qp, dt, s));
 }
 
@@ -367,7 +362,7 @@ ba_status forward(const void* q, const void* k, const void* v, ba_dtype dt, int 
     record(ev, 2, s);
     record(ev, 3, s);
   } else {
-    // One launch streams q, k and v: sign bits + |x| partial sums for q and k, channel
+    // One launch streams q, k and v: sign bits + |x| partial sums for q and k, partial channel
     // maxima for v.
     PrepParams pp{};
     pp.g = g;
@@ -376,23 +371,20 @@ ba_status forward(const void* q, const void* k, const void* v, ba_dtype dt, int 
     pp.job[2] = PrepJob{v, kJobAmax, nullptr, nullptr, at<float>(ws, L.part_amax)};
     if ((st = cuda_status(launch_prep(pp, dt, 3, s))) != BA_OK) return keep(ev, false), st;
     record(ev, 1, s);
-    FinalizeParams fp{};
-    fp.g = g;
-    fp.npack = 2;
-    fp.part_mu[0] = at<double>(ws, L.part_mu_q);
-    fp.part_mu[1] = at<double>(ws, L.part_mu_k);
-    fp.mu[0] = at<float>(ws, L.mu_q);
-    fp.mu[1] = at<float>(ws, L.mu_k);
-    fp.part_amax = at<float>(ws, L.part_amax);
-    fp.inv = at<float>(ws, L.inv);
-    fp.v_scale = at<float>(ws, L.v_scale);
-    if ((st = cuda_status(launch_finalize(fp, s))) != BA_OK) return keep(ev, false), st;
-    record(ev, 2, s);
+    record(ev, 2, s);  // the finalize is folded into the quantiser
+    // The quantiser reduces the V partials to scales and writes int8 V and mu of q and k.
     QuantParams qp{};
     qp.g = g;
     qp.v = v;
-    qp.inv = at<float>(ws, L.inv);
+    qp.part_amax = at<float>(ws, L.part_amax);
+    qp.npart = amax_parts(g);
+    qp.v_scale = at<float>(ws, L.v_scale);
     qp.vq = at<int8_t>(ws, L.vq);
+    qp.npack = 2;
+    qp.part_mu[0] = at<double>(ws, L.part_mu_q);
+    qp.part_mu[1] = at<double>(ws, L.part_mu_k);
+    qp.mu[0] = at<float>(ws, L.mu_q);
+    qp.mu[1] = at<float>(ws, L.mu_k);
     if ((st = cuda_status(launch_quant(qp, dt, s))) != BA_OK) return keep(ev, false), st;
     record(ev, 3, s);
   }

@@ -9,7 +9,8 @@
 namespace binattn {
 
 constexpr int kJobPack = 0;  // sign bits + sum |x| per chunk
-constexpr int kJobAmax = 1;  // per-channel max |v| per chunk
+constexpr int kJobAmax = 1;  // per-channel max |v| per group of chunks
+constexpr int kQuantTokens = 1024;  // tokens per CTA of the V quantiser
 
 struct PrepDims {
   int64_t BH;
@@ -21,7 +22,7 @@ struct PrepJob {
   int kind;
   uint32_t* bits;    // pack: [BH][N][4]
   double* part_sum;  // pack: [BH][nchunk] sums of |x|
-  float* part;       // amax: [BH][nchunk][dp] channel maxima
+  float* part;       // amax: [BH][amax_parts][dp] channel maxima
 };
 
 struct PrepParams {
@@ -29,21 +30,27 @@ struct PrepParams {
   PrepDims g;
 };
 
+// mu = sum |x| / (N d) per slice from the per-chunk partial sums (standalone sign packing).
 struct FinalizeParams {
   PrepDims g;
   int npack;
   const double* part_mu[2];
   float* mu[2];
-  const float* part_amax;  // null: no V job
-  float* inv;              // [BH][dp]
-  float* v_scale;          // [BH][d]
 };
 
+// V quantiser with the finalize folded in: each CTA reduces its slice's partial channel maxima
+// (npart rows of dp floats), then writes int8 rows for kQuantTokens tokens; a slice's first CTA
+// also writes the V scales and the mu of up to two packed tensors from their chunk sums.
 struct QuantParams {
   PrepDims g;
   const void* v;
-  const float* inv;
-  int8_t* vq;
+  const float* part_amax;  // [BH][npart][dp]
+  int npart;
+  float* v_scale;  // [BH][d]
+  int8_t* vq;      // [BH][N][dp]
+  int npack;
+  const double* part_mu[2];  // [BH][nchunk]
+  float* mu[2];              // [BH]
 };
 
 // Whole-slice preparation (one warp per (b, h) and tensor; d % 8 == 0): sign bits and mu of q
@@ -61,9 +68,11 @@ struct SliceParams {
   float* v_scale;
 };
 
+// Jobs [0, njobs): the sign-packing jobs first, then at most one channel-max job.
 cudaError_t launch_prep(const PrepParams& p, int dt, int njobs, cudaStream_t s);
 cudaError_t launch_prep_slices(const SliceParams& p, int dt, cudaStream_t s);
 bool use_slice_prep(const PrepDims& g);
+int amax_parts(const PrepDims& g);  // partial channel-max rows per slice written by launch_prep
 cudaError_t launch_finalize(const FinalizeParams& p, cudaStream_t s);
 cudaError_t launch_quant(const QuantParams& p, int dt, cudaStream_t s);
 

@@ -3,10 +3,13 @@
 //                       tensor) writes the sign bits and mu of q and k, or the scales and int8
 //                       rows of v, in one launch;
 //   prep_warp_kernel  — otherwise, rows of whole 16-byte pieces: one warp per 128-token chunk,
-//                       sign bits + per-chunk sum |x| of q and k, per-chunk channel max |v|;
-//   prep_kernel       — the same per chunk for any d (CTA per chunk; scalar path when d % 8 != 0);
-//   finalize_kernel   — mu = sum / (N d) per (b, h); per-channel V scales;
-//   quant_kernel      — V -> int8 rows with the per-channel inverse scale.
+//                       sign bits + per-chunk sum |x| of q and k; one CTA per eight chunks of
+//                       v, their channel max |v|;
+//   prep_kernel       — d % 8 != 0: a CTA per (tensor, chunk), the same per-chunk partials;
+//   quant_kernel      — V -> int8 rows, 1024 tokens per CTA; each CTA reduces its slice's
+//                       channel-max partials to the inverse scales itself, and a slice's first
+//                       CTA writes mu of q and k and the V scales (no separate finalize launch);
+//   finalize_kernel   — mu = sum / (N d) per (b, h), for sign packing on its own.
 // Sign binarisation and mu: gist.science/zh technical summary 2.2(1) (s_i = mu_q sign(q_i),
 // mu the mean along token and channel axes). Channel-aware 8-bit V: gist.science/zh 2.2(3),
 // gist.science/nl Methodologie 2.
@@ -25,7 +28,6 @@ namespace binattn {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kMaxIter = 8;  // ceil(kPrepTokens / rows_per_pass) for d/8 <= 16
 
 // Sum over the CTA in double. Every |x| of a 16-bit input is exact in double and the
 // partial sums stay exact while they are below 2^53 units of the smallest input's ulp, so
@@ -42,91 +44,6 @@ __device__ __forceinline__ double block_sum(double v, double* sred) {
     for (int w = 0; w < kThreads / 32; ++w) t += sred[w];
   }
   return t;  // valid in thread 0
-}
-
-// Vector path: d % 8 == 0, so every row is a whole number of 16-byte pieces.
-template <typename T>
-__device__ void prep_pack_vec(const PrepJob& job, const PrepDims& g, int64_t bh, int chunk) {
-  __shared__ __align__(16) uint8_t sbits[kPrepTokens][16];
-  __shared__ double sred[kThreads / 32];
-  const int tok0 = chunk * kPrepTokens;
-  const int ntok = min(kPrepTokens, g.N - tok0);
-  const int tpr = g.d >> 3;
-  const int rpp = kThreads / tpr;
-  const int sub = threadIdx.x % tpr, r0 = threadIdx.x / tpr;
-  reinterpret_cast<uint2*>(&sbits[0][0])[threadIdx.x] = make_uint2(0u, 0u);
-  __syncthreads();
-  const char* base = reinterpret_cast<const char*>(job.src) + ((bh * g.N + tok0) * g.d) * 2;
-  uint4 u[kMaxIter];
-#pragma unroll
-  for (int it = 0; it < kMaxIter; ++it) {
-    const int r = r0 + it * rpp;
-    if (r0 < rpp && r < ntok) u[it] = ldg_stream(base + (static_cast<int64_t>(r) * g.d + sub * 8) * 2);
-  }
-  double acc = 0.0;
-#pragma unroll
-  for (int it = 0; it < kMaxIter; ++it) {
-    const int r = r0 + it * rpp;
-    if (r0 < rpp && r < ntok) {
-      float f[8];
-      unpack8<T>(u[it], f);
-      uint32_t byte = 0;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        byte |= (f[e] < 0.0f ? 1u : 0u) << e;
-        acc += static_cast<double>(fabsf(f[e]));
-      }
-      sbits[r][sub] = static_cast<uint8_t>(byte);
-    }
-  }
-  __syncthreads();
-  if (threadIdx.x < ntok)
-    reinterpret_cast<uint4*>(job.bits)[bh * g.N + tok0 + threadIdx.x] =
-        reinterpret_cast<const uint4*>(&sbits[0][0])[threadIdx.x];
-  const double tot = block_sum(acc, sred);
-  if (threadIdx.x == 0) job.part_sum[bh * g.nchunk + chunk] = tot;
-}
-
-template <typename T>
-__device__ void prep_amax_vec(const PrepJob& job, const PrepDims& g, int64_t bh, int chunk) {
-  __shared__ float sred[kThreads * 8];
-  const int tok0 = chunk * kPrepTokens;
-  const int ntok = min(kPrepTokens, g.N - tok0);
-  const int tpr = g.d >> 3;
-  const int rpp = kThreads / tpr;
-  const int sub = threadIdx.x % tpr, r0 = threadIdx.x / tpr;
-  const char* base = reinterpret_cast<const char*>(job.src) + ((bh * g.N + tok0) * g.d) * 2;
-  uint4 u[kMaxIter];
-#pragma unroll
-  for (int it = 0; it < kMaxIter; ++it) {
-    const int r = r0 + it * rpp;
-    if (r0 < rpp && r < ntok) u[it] = ldg_stream(base + (static_cast<int64_t>(r) * g.d + sub * 8) * 2);
-  }
-  float mx[8];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) mx[e] = 0.0f;
-#pragma unroll
-  for (int it = 0; it < kMaxIter; ++it) {
-    const int r = r0 + it * rpp;
-    if (r0 < rpp && r < ntok) {
-      float f[8];
-      unpack8<T>(u[it], f);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) mx[e] = fmaxf(mx[e], fabsf(f[e]));
-    }
-  }
-  if (r0 < rpp) {
-#pragma unroll
-    for (int e = 0; e < 8; ++e) sred[r0 * g.d + sub * 8 + e] = mx[e];
-  }
-  __syncthreads();
-  const int rows = min(rpp, ntok);
-  for (int c = threadIdx.x; c < g.dp; c += kThreads) {
-    float m = 0.0f;
-    if (c < g.d)
-      for (int rr = 0; rr < rows; ++rr) m = fmaxf(m, sred[rr * g.d + c]);
-    job.part[(bh * g.nchunk + chunk) * g.dp + c] = m;
-  }
 }
 
 // Scalar path for d % 8 != 0 (rows not made of whole 16-byte pieces).
@@ -171,14 +88,7 @@ __global__ void __launch_bounds__(kThreads) prep_kernel(PrepParams p) {
   const int64_t bh = cta / p.g.nchunk;
   const int chunk = static_cast<int>(cta - bh * p.g.nchunk);
   const PrepJob job = (blockIdx.y == 0) ? p.job[0] : (blockIdx.y == 1 ? p.job[1] : p.job[2]);
-  if ((p.g.d & 7) == 0) {
-    if (job.kind == kJobPack)
-      prep_pack_vec<T>(job, p.g, bh, chunk);
-    else
-      prep_amax_vec<T>(job, p.g, bh, chunk);
-  } else {
-    prep_scalar<T>(job, p.g, bh, chunk);
-  }
+  prep_scalar<T>(job, p.g, bh, chunk);
 }
 
 // A channel gets codes when its maximum is nonzero and 127 / amax is a finite float. A bf16
@@ -188,28 +98,15 @@ __device__ __forceinline__ bool channel_live(float amax, float inv) {
   return amax > 0.0f && inv <= 3.402823466e38f;
 }
 
-__global__ void __launch_bounds__(128) finalize_kernel(FinalizeParams p) {
+__global__ void __launch_bounds__(32) finalize_kernel(FinalizeParams p) {
   const int64_t bh = blockIdx.x;
   const PrepDims& g = p.g;
-  if (threadIdx.x < 32) {
-    for (int j = 0; j < p.npack; ++j) {
-      // Fixed-order double sum of the chunk partials.
-      double s = 0.0;
-      for (int c = threadIdx.x; c < g.nchunk; c += 32) s += p.part_mu[j][bh * g.nchunk + c];
+  for (int j = 0; j < p.npack; ++j) {
+    double s = 0.0;
+    for (int c = threadIdx.x; c < g.nchunk; c += 32) s += p.part_mu[j][bh * g.nchunk + c];
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-      if (threadIdx.x == 0) p.mu[j][bh] = static_cast<float>(s / (static_cast<double>(g.N) * g.d));
-    }
-  }
-  if (p.part_amax != nullptr) {
-    for (int c = threadIdx.x; c < g.dp; c += blockDim.x) {
-      float m = 0.0f;
-      for (int ch = 0; ch < g.nchunk; ++ch) m = fmaxf(m, p.part_amax[(bh * g.nchunk + ch) * g.dp + c]);
-      const float inv = __fdiv_rn(127.0f, m);
-      const bool live = (c < g.d) && channel_live(m, inv);
-      p.inv[bh * g.dp + c] = live ? inv : 0.0f;
-      if (c < g.d) p.v_scale[bh * g.d + c] = live ? __fdiv_rn(m, 127.0f) : 0.0f;
-    }
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (threadIdx.x == 0) p.mu[j][bh] = static_cast<float>(s / (static_cast<double>(g.N) * g.d));
   }
 }
 
@@ -225,43 +122,122 @@ __device__ __forceinline__ uint32_t quant4(const float* f, const float* inv) {
   return __byte_perm(__byte_perm(y[0], y[1], 0x0040), __byte_perm(y[2], y[3], 0x0040), 0x5410);
 }
 
+constexpr int kQuantBatch = 8;  // passes of the quantiser whose loads are in flight together
+
+// Loads of one batch of V pieces: row r0 + j rpp + rp, piece sub, for j < kQuantBatch.
+__device__ __forceinline__ void quant_load(uint4 (&u)[kQuantBatch], const char* base, int r0, int ntok, int d,
+                                           int rpp, int rp, int sub, bool on) {
+#pragma unroll
+  for (int j = 0; j < kQuantBatch; ++j) {
+    const int r = r0 + j * rpp + rp;
+    if (on && r < ntok) u[j] = ldg_stream(base + (static_cast<int64_t>(r) * d + sub * 8) * 2);
+  }
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kThreads) quant_kernel(QuantParams p) {
   allow_dependents();  // the attention kernel may start early; it waits for this grid
+  __shared__ float4 sred[kThreads];
   __shared__ float sinv[128];
-  const int64_t cta = blockIdx.x;
-  const int64_t bh = cta / p.g.nchunk;
-  const int chunk = static_cast<int>(cta - bh * p.g.nchunk);
-  const int tok0 = chunk * kPrepTokens;
-  const int ntok = min(kPrepTokens, p.g.N - tok0);
-  const int d = p.g.d, dp = p.g.dp;
-  if (threadIdx.x < dp) sinv[threadIdx.x] = p.inv[bh * dp + threadIdx.x];
-  __syncthreads();
-  int8_t* out = p.vq + (bh * p.g.N + tok0) * dp;
-  if ((d & 7) == 0) {
-    const int opr = dp >> 3;  // 8-byte output pieces per row
-    const int rpp = kThreads / opr;
-    const int sub = threadIdx.x % opr, r0 = threadIdx.x / opr;
-    if (r0 >= rpp) return;
-    const char* base = reinterpret_cast<const char*>(p.v) + ((bh * p.g.N + tok0) * d) * 2;
-    for (int r = r0; r < ntok; r += rpp) {
-      uint2 w = make_uint2(0u, 0u);
-      if (sub * 8 < d) {
-        const uint4 u = ldg_stream(base + (static_cast<int64_t>(r) * d + sub * 8) * 2);
-        float f[8];
-        unpack8<T>(u, f);
-        w.x = quant4(f, &sinv[sub * 8]);
-        w.y = quant4(f + 4, &sinv[sub * 8 + 4]);
+  const PrepDims& g = p.g;
+  const int d = g.d, dp = g.dp;
+  const int ngrp = (g.N + kQuantTokens - 1) / kQuantTokens;
+  // Last slice first: the streaming kernel before this one reads V in slice order, so the
+  // slices it read last are the likeliest to be still in L2.
+  const int64_t cta = static_cast<int64_t>(gridDim.x) - 1 - blockIdx.x;
+  const int64_t bh = cta / ngrp;
+  const int grp = static_cast<int>(cta - bh * ngrp);
+  const int tok0 = grp * kQuantTokens;
+  const int ntok = min(kQuantTokens, g.N - tok0);
+  const bool vec = (d & 7) == 0;
+  // Vector path: thread (rp, sub) writes the 8-byte piece sub of rows rp + rpp t; pieces at or
+  // past d are the zero padding of the row.
+  const int opr = dp >> 3;
+  const int rpp = kThreads / opr;
+  const int sub = threadIdx.x % opr, rp = threadIdx.x / opr;
+  const bool on_row = vec && rp < rpp;
+  const bool on = on_row && sub * 8 < d;
+  const char* base = reinterpret_cast<const char*>(p.v) + ((bh * g.N + tok0) * d) * 2;
+  // The first batch reads only the caller's V: it is in flight while this CTA waits for the
+  // streaming kernel's partials.
+  uint4 u[kQuantBatch];
+  quant_load(u, base, 0, ntok, d, rpp, rp, sub, on);
+  grid_dependency_wait();
+
+  // Channel maxima of the slice: the max over its npart partial rows, read as float4 columns by
+  // rstride row lanes each, then over the row lanes in shared memory.
+  const int nc4 = dp >> 2;
+  const int rstride = kThreads / nc4;
+  {
+    const int col = threadIdx.x % nc4, r0 = threadIdx.x / nc4;
+    float4 m = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    if (r0 < rstride) {
+      const float4* src = reinterpret_cast<const float4*>(p.part_amax + bh * p.npart * dp) + col;
+#pragma unroll 4
+      for (int r = r0; r < p.npart; r += rstride) {
+        const float4 x = __ldcg(src + static_cast<int64_t>(r) * nc4);
+        m.x = fmaxf(m.x, x.x);
+        m.y = fmaxf(m.y, x.y);
+        m.z = fmaxf(m.z, x.z);
+        m.w = fmaxf(m.w, x.w);
       }
-      *reinterpret_cast<uint2*>(out + static_cast<int64_t>(r) * dp + sub * 8) = w;
+    }
+    sred[threadIdx.x] = m;
+  }
+  __syncthreads();
+  if (threadIdx.x < dp) {
+    const int c = threadIdx.x;
+    const float* sr = reinterpret_cast<const float*>(sred);
+    float m = 0.0f;
+    for (int rr = 0; rr < rstride; ++rr) m = fmaxf(m, sr[rr * dp + c]);
+    const float inv = __fdiv_rn(127.0f, m);
+    const bool live = (c < d) && channel_live(m, inv);
+    sinv[c] = live ? inv : 0.0f;
+    if (grp == 0 && c < d) p.v_scale[bh * d + c] = live ? __fdiv_rn(m, 127.0f) : 0.0f;
+  }
+  // mu of the packed tensors (one warp each, on the slice's first CTA): the sum of the chunk
+  // partials, exact in double in any order, over N d.
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (grp == 0 && warp < p.npack) {
+    const double* src = (warp == 0 ? p.part_mu[0] : p.part_mu[1]) + bh * g.nchunk;
+    double s = 0.0;
+    for (int c = lane; c < g.nchunk; c += 32) s += __ldcg(src + c);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (lane == 0) (warp == 0 ? p.mu[0] : p.mu[1])[bh] = static_cast<float>(s / (static_cast<double>(g.N) * d));
+  }
+  __syncthreads();
+
+  int8_t* out = p.vq + (bh * g.N + tok0) * dp;
+  if (vec) {
+    float inv[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) inv[e] = sinv[sub * 8 + e];
+    const int rows_per_batch = kQuantBatch * rpp;
+    for (int r0 = 0; r0 < ntok; r0 += rows_per_batch) {
+      if (r0 > 0) quant_load(u, base, r0, ntok, d, rpp, rp, sub, on);
+#pragma unroll
+      for (int j = 0; j < kQuantBatch; ++j) {
+        const int r = r0 + j * rpp + rp;
+        if (on_row && r < ntok) {
+          uint2 w = make_uint2(0u, 0u);
+          if (on) {
+            float f[8];
+            unpack8<T>(u[j], f);
+            w.x = quant4(f, inv);
+            w.y = quant4(f + 4, inv + 4);
+          }
+          *reinterpret_cast<uint2*>(out + static_cast<int64_t>(r) * dp + sub * 8) = w;
+        }
+      }
     }
   } else {
-    const T* base = reinterpret_cast<const T*>(p.v) + (bh * p.g.N + tok0) * d;
+    const T* vb = reinterpret_cast<const T*>(p.v) + (bh * g.N + tok0) * d;
     for (int e = threadIdx.x; e < ntok * dp; e += kThreads) {
       const int r = e / dp, c = e - r * dp;
       int q = 0;
       if (c < d) {
-        q = __float2int_rn(__fmul_rn(load1<T>(base + static_cast<int64_t>(r) * d + c), sinv[c]));
+        q = __float2int_rn(__fmul_rn(load1<T>(vb + static_cast<int64_t>(r) * d + c), sinv[c]));
         q = max(-127, min(127, q));
       }
       out[e] = static_cast<int8_t>(q);
@@ -436,40 +412,60 @@ __device__ __forceinline__ uint8_t (*warp_bits_rows())[16] {
   return sb;
 }
 
-// Chunk mode: one warp per (job, slice, 128-token chunk); per-chunk partials for finalize.
+// Chunk mode. CTAs [0, pack_ctas): one warp per (packing job, slice, 128-token chunk), its sign
+// rows and partial sum |x|. The CTAs after them (when there is a channel-max job): one per
+// (slice, group of kWarps chunks), a warp per chunk, the group's channel maxima reduced in
+// shared memory to one partial row. The V CTAs come last in the grid, so V is the tensor read
+// most recently when the quantiser reads it again.
 template <typename T>
-__global__ void __launch_bounds__(kThreads, 3) prep_warp_kernel(PrepParams p, int njobs) {
+__global__ void __launch_bounds__(kThreads, 3) prep_warp_kernel(PrepParams p, int npack, unsigned pack_ctas) {
+  allow_dependents();  // the quantiser may start early; it waits for this grid
   const PrepDims& g = p.g;
-  const int64_t per_job = g.BH * g.nchunk;
-  const int64_t unit = static_cast<int64_t>(blockIdx.x) * kWarps + (threadIdx.x >> 5);
-  uint8_t (*sb)[16] = warp_bits_rows();
-  if (unit >= njobs * per_job) return;
-  const int j = static_cast<int>(unit / per_job);
-  const PrepJob job = j == 0 ? p.job[0] : (j == 1 ? p.job[1] : p.job[2]);
-  const int64_t rest = unit - j * per_job;
-  const int64_t bh = rest / g.nchunk;
-  const int chunk = static_cast<int>(rest - bh * g.nchunk);
-  const int tok0 = chunk * kPrepTokens;
-  const int ntok = min(kPrepTokens, g.N - tok0);
   const Lanes L = lanes_for(g.d);
-  const char* rows = reinterpret_cast<const char*>(job.src) + ((bh * g.N + tok0) * g.d) * 2;
-  if (job.kind == kJobPack) {
+  const int warp = threadIdx.x >> 5;
+  if (blockIdx.x < pack_ctas) {
+    const int64_t per_job = g.BH * g.nchunk;
+    const int64_t unit = static_cast<int64_t>(blockIdx.x) * kWarps + warp;
+    uint8_t (*sb)[16] = warp_bits_rows();
+    if (unit >= npack * per_job) return;
+    const int j = static_cast<int>(unit / per_job);
+    const PrepJob job = j == 0 ? p.job[0] : p.job[1];
+    const int64_t rest = unit - j * per_job;
+    const int64_t bh = rest / g.nchunk;
+    const int chunk = static_cast<int>(rest - bh * g.nchunk);
+    const int tok0 = chunk * kPrepTokens;
+    const int ntok = min(kPrepTokens, g.N - tok0);
+    const char* rows = reinterpret_cast<const char*>(job.src) + ((bh * g.N + tok0) * g.d) * 2;
     const double tot = warp_sum(pack_chunk<T>(rows, ntok, g.d, L, sb, reinterpret_cast<uint4*>(job.bits) + bh * g.N + tok0));
     if ((threadIdx.x & 31) == 0) job.part_sum[bh * g.nchunk + chunk] = tot;
-  } else {
-    float mx[8];
+    return;
+  }
+  __shared__ float smax[kWarps][128];
+  const PrepJob job = npack == 0 ? p.job[0] : (npack == 1 ? p.job[1] : p.job[2]);
+  const int ngrp = (g.nchunk + kWarps - 1) / kWarps;
+  const int64_t c = blockIdx.x - pack_ctas;
+  const int64_t bh = c / ngrp;
+  const int grp = static_cast<int>(c - bh * ngrp);
+  const int chunk = grp * kWarps + warp;
+  float mx[8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) mx[e] = 0.0f;
-    amax_chunk<T>(rows, ntok, g.d, L, mx);
-    group_max(mx, L);
-    if (L.on && L.rp == 0) {
-      float* out = job.part + (bh * g.nchunk + chunk) * g.dp + L.sub * 8;
+  for (int e = 0; e < 8; ++e) mx[e] = 0.0f;
+  if (chunk < g.nchunk) {
+    const int tok0 = chunk * kPrepTokens;
+    const int ntok = min(kPrepTokens, g.N - tok0);
+    amax_chunk<T>(reinterpret_cast<const char*>(job.src) + ((bh * g.N + tok0) * g.d) * 2, ntok, g.d, L, mx);
+  }
+  group_max(mx, L);
+  if (L.on && L.rp == 0) {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) out[e] = mx[e];
-      if ((g.d & 15) == 8 && L.sub == L.tpr - 1)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) out[8 + e] = 0.0f;
-    }
+    for (int e = 0; e < 8; ++e) smax[warp][L.sub * 8 + e] = mx[e];
+  }
+  __syncthreads();
+  for (int ch = threadIdx.x; ch < g.dp; ch += kThreads) {
+    float m = 0.0f;
+    if (ch < g.d)
+      for (int w = 0; w < kWarps; ++w) m = fmaxf(m, smax[w][ch]);
+    job.part[(bh * ngrp + grp) * g.dp + ch] = m;
   }
 }
 
@@ -625,13 +621,18 @@ __global__ void __launch_bounds__(kThreads, kSliceBatch <= kSliceBatchShort ? 4 
 
 unsigned warp_grid(int64_t units) { return static_cast<unsigned>(ceil_div(units, kWarps)); }
 
+int amax_parts(const PrepDims& g) { return (g.d & 7) == 0 ? static_cast<int>(ceil_div(g.nchunk, kWarps)) : g.nchunk; }
+
 cudaError_t launch_prep(const PrepParams& p, int dt, int njobs, cudaStream_t s) {
   if ((p.g.d & 7) == 0) {
-    const unsigned grid = warp_grid(njobs * p.g.BH * p.g.nchunk);
+    int npack = 0;
+    while (npack < njobs && p.job[npack].kind == kJobPack) ++npack;
+    const unsigned pack_ctas = warp_grid(npack * p.g.BH * p.g.nchunk);
+    const unsigned grid = pack_ctas + (npack < njobs ? static_cast<unsigned>(p.g.BH * amax_parts(p.g)) : 0u);
     if (dt == BA_F16)
-      prep_warp_kernel<__half><<<grid, kThreads, 0, s>>>(p, njobs);
+      prep_warp_kernel<__half><<<grid, kThreads, 0, s>>>(p, npack, pack_ctas);
     else
-      prep_warp_kernel<__nv_bfloat16><<<grid, kThreads, 0, s>>>(p, njobs);
+      prep_warp_kernel<__nv_bfloat16><<<grid, kThreads, 0, s>>>(p, npack, pack_ctas);
     return cudaGetLastError();
   }
   const dim3 grid(static_cast<unsigned>(p.g.BH * p.g.nchunk), static_cast<unsigned>(njobs));
@@ -643,7 +644,7 @@ cudaError_t launch_prep(const PrepParams& p, int dt, int njobs, cudaStream_t s) 
 }
 
 cudaError_t launch_finalize(const FinalizeParams& p, cudaStream_t s) {
-  finalize_kernel<<<static_cast<unsigned>(p.g.BH), 128, 0, s>>>(p);
+  finalize_kernel<<<static_cast<unsigned>(p.g.BH), 32, 0, s>>>(p);
   return cudaGetLastError();
 }
 
@@ -674,13 +675,21 @@ cudaError_t launch_prep_slices(const SliceParams& p, int dt, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+// A programmatic dependent of the streaming kernel: its CTAs may be resident, with their first
+// V loads in flight, before that grid completes.
 cudaError_t launch_quant(const QuantParams& p, int dt, cudaStream_t s) {
-  const unsigned grid = static_cast<unsigned>(p.g.BH * p.g.nchunk);
-  if (dt == BA_F16)
-    quant_kernel<__half><<<grid, kThreads, 0, s>>>(p);
-  else
-    quant_kernel<__nv_bfloat16><<<grid, kThreads, 0, s>>>(p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(p.g.BH * ceil_div(p.g.N, kQuantTokens)));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (dt == BA_F16) return cudaLaunchKernelEx(&cfg, quant_kernel<__half>, p);
+  return cudaLaunchKernelEx(&cfg, quant_kernel<__nv_bfloat16>, p);
 }
 
 }  // namespace binattn
