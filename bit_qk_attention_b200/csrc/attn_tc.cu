@@ -74,14 +74,22 @@ __host__ __device__ constexpr bool is_relpos_general(int bk) { return bk == kRel
 
 template <int DP, int BK>
 struct Cfg {
-  // One 128-row query tile per item and CTA, S double-buffered (QK of the next block runs while
-  // the softmax works on this one). Two tiles with one S buffer each also fit tensor memory for
-  // heads up to 64 channels, but their 640 threads leave the softmax too few registers.
-  static constexpr int NQ = 1;                 // query tiles per item
-  static constexpr int SB = NQ == 1 ? 2 : 1;   // S buffers per tile
+  // Heads up to 64 channels: two 128-row query tiles per item, one S buffer each; softmax
+  // warpgroup q owns tile q (the tiles ping-pong: one's MMAs run while the other's softmax
+  // works). Wider heads: one tile, S double-buffered, the two softmax warpgroups taking
+  // alternate key blocks (the blocks ping-pong).
+  static constexpr bool kTilePP = DP <= 64;
+  static constexpr int NQ = kTilePP ? 2 : 1;   // query tiles per item
+  static constexpr int SB = kTilePP ? 1 : 2;   // S buffers per tile
   static constexpr int DQ = (DP + 31) / 32 * 32;  // QK contraction width: fp8 K-steps of 32
   static constexpr int DH = DP / 2;            // accumulator / output columns per softmax half
-  static constexpr int kThreads = 128 + 256 * NQ;
+  static constexpr int kThreads = 384;  // 4 service warps, 2 softmax warpgroups
+  // Service warps: warp 0 V copies and bias data, warp 1 issues the MMAs (of both tiles, when
+  // there are two), warps 2 and 3 expand the sign rows. (One MMA warp per tile, with one
+  // expanding warp, measured 5-20 % slower on d = 64 heads.)
+  static constexpr int kExpWarps = 2;
+  static constexpr int kMmaWarps = 1;
+  static constexpr int kRowsPerLane = BM / (32 * kExpWarps);  // sign rows a lane expands per tile
   static constexpr int kStages = 4;
   static constexpr int kQBytes = BM * DQ;
   static constexpr int kKBytes = BN * DQ;
@@ -95,8 +103,8 @@ struct Cfg {
   static constexpr int offWin = offV + kStages * kVBytes;  // [S][NQ][kWinFloats] f32
   static constexpr int offWinK = offWin + kWinBytes;       // [S][NQ][4] s32 chunk offsets
   static constexpr int offKoff = offWinK + kWinKBytes;     // [S][BN] s32 key offsets
-  static constexpr int offX = offKoff + kKoffBytes;        // per row: m_j [2][BM], L' [BM], m_ref [BM]
-  static constexpr int offBar = offX + 4 * BM * 4;
+  static constexpr int offX = offKoff + kKoffBytes;  // per row: m_j [2][BM]; (L', m_ref) [2][BM]
+  static constexpr int offBar = offX + 2 * BM * 4 + 2 * BM * 8;
   static constexpr int kNumBars = 2 * kStages + 3 + 2 + 2 + 2 + 2 + 1 + 4;
   static constexpr int offMisc = offBar + kNumBars * 8;  // tmem base, abort flag
   static constexpr int kBytes = offMisc + 16;
@@ -104,7 +112,8 @@ struct Cfg {
   // Tensor-memory columns of tile q: S buffer b (fp32, 128 columns; the softmax overwrites its
   // first 32 columns with the uint8 codes P — the MMAs of one CTA run in issue order, so P.V
   // reads P before the next QK into that buffer rewrites it), the s32 P.V accumulator of one
-  // block (DP) and the fp32 running output F' (DP).
+  // block (DP) and the fp32 running output F' (DP): 256 columns per tile for two tiles, or
+  // 2 x 128 + 2 DP for one.
   __host__ __device__ static constexpr uint32_t tS(int q, int b) { return q * 256 + b * 128; }
   __host__ __device__ static constexpr uint32_t tAcc(int q) { return q * 256 + SB * 128; }
   __host__ __device__ static constexpr uint32_t tF(int q) { return tAcc(q) + DP; }
@@ -133,7 +142,7 @@ struct Bars {
   __host__ __device__ static constexpr int folddone(int g) { return 2 * S + 9 + g; }
   __host__ __device__ static constexpr int epidone() { return 2 * S + 11; }
   __host__ __device__ static constexpr int mchain(int w4) { return 2 * S + 12 + w4; }
-  static_assert(NQ == 1 && SB == 2, "one tile, two S buffers");
+  static_assert(NQ * SB == 2, "two S buffers: one per tile, or two for one tile");
   static_assert(mchain(3) + 1 == C::kNumBars, "barrier count");
 };
 
@@ -297,14 +306,16 @@ __global__ void __launch_bounds__(Cfg<DP, BK>::kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int st = 0; st < S; ++st) {
-      // kv_full: the V copy's expect_tx arrival + warp 0 (bias data) + the two expanding warps.
-      mbar_init(&bars[Bar::kvfull(st)], 4);
-      mbar_init(&bars[Bar::kvempty(st)], 1);
+      // kv_full: the V copy's expect_tx arrival + warp 0 (bias data) + the expanding warps;
+      // kv_empty: one commit per MMA-issuing warp.
+      mbar_init(&bars[Bar::kvfull(st)], 2 + C::kExpWarps);
+      mbar_init(&bars[Bar::kvempty(st)], C::kMmaWarps);
     }
-    mbar_init(&bars[Bar::qfull()], 2);
-    mbar_init(&bars[Bar::qempty()], 1);
-    mbar_init(&bars[Bar::drain()], 1);
-    for (int b = 0; b < SB; ++b) mbar_init(&bars[Bar::sfull(0, b)], 1);
+    mbar_init(&bars[Bar::qfull()], C::kExpWarps);
+    mbar_init(&bars[Bar::qempty()], C::kMmaWarps);
+    mbar_init(&bars[Bar::drain()], C::kMmaWarps);
+    for (int q = 0; q < NQ; ++q)
+      for (int b = 0; b < SB; ++b) mbar_init(&bars[Bar::sfull(q, b)], 1);
     for (int g = 0; g < 2; ++g) mbar_init(&bars[Bar::pfull(g)], 4);  // the group's four warps
     for (int g = 0; g < 2; ++g) {
       mbar_init(&bars[Bar::pvdone(g)], 1);
@@ -435,16 +446,21 @@ __global__ void __launch_bounds__(Cfg<DP, BK>::kThreads, 1)
     // Leave no TMA copy in flight: wait (bounded, even after an abort) for the stages this
     // warp filled last.
     for (int k = (g > S ? g - S : 0); k < g; ++k) wait_bounded(&bars[Bar::kvfull(k % S)], (k / S) & 1, abort_flag, false);
-  } else if (warp == 2 || warp == 3) {
+  } else if (warp < 4 && warp >= 4 - C::kExpWarps) {
     // ------------------------------------------------------------ producer: sign expansion
-    // Warp 2 expands rows 0..63 and warp 3 rows 64..127 of every Q tile and K block. The sign
-    // rows of the next K block are loaded into registers before this block is written. The Q
-    // tiles of an item are written once the MMAs of the previous item have read them (q_empty).
-    const int half = warp - 2;
+    // The expanding warps split the 128 rows of every Q tile and K block (warp 2 rows 0..63 and
+    // warp 3 rows 64..127). The sign rows of the next K block are loaded
+    // into registers before this block is written. The Q tiles of an item are written once the
+    // MMAs of the previous item have read them (q_empty).
+    constexpr int RPL = C::kRowsPerLane;
+    const int half = warp - (4 - C::kExpWarps);
+    const int rbase = half * (BM / C::kExpWarps);
     int g = 0;
     bool ok = true;
-    uint4 nb[2] = {zero4, zero4};
-    uint4 pre_q[NQ][2];
+    uint4 nb[RPL];
+#pragma unroll
+    for (int u = 0; u < RPL; ++u) nb[u] = zero4;
+    uint4 pre_q[NQ][RPL];
     for (int it = 0; it < n_items && ok; ++it) {
       int64_t bh;
       int q0;
@@ -453,15 +469,15 @@ __global__ void __launch_bounds__(Cfg<DP, BK>::kThreads, 1)
 #pragma unroll
       for (int q = 0; q < NQ; ++q)
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int row = q0 + q * BM + 64 * half + lane + 32 * u;
+        for (int u = 0; u < RPL; ++u) {
+          const int row = q0 + q * BM + rbase + lane + 32 * u;
           pre_q[q][u] = row < N ? __ldg(qrows + row) : zero4;
         }
       if (it == 0) {
         const uint4* krows = reinterpret_cast<const uint4*>(p.bits_k) + bh * N;
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int row = 64 * half + lane + 32 * u;
+        for (int u = 0; u < RPL; ++u) {
+          const int row = rbase + lane + 32 * u;
           nb[u] = row < N ? __ldg(krows + row) : zero4;
         }
       } else if (!wait_warp(&bars[Bar::qempty()], (it - 1) & 1, abort_flag)) {
@@ -470,15 +486,17 @@ __global__ void __launch_bounds__(Cfg<DP, BK>::kThreads, 1)
 #pragma unroll
       for (int q = 0; q < NQ; ++q)
 #pragma unroll
-        for (int u = 0; u < 2; ++u)
-          expand_row<DQ>(sQ + q * C::kQBytes, pre_q[q][u], q0 + q * BM + 64 * half + lane + 32 * u < N,
-                         64 * half + lane + 32 * u, d);
+        for (int u = 0; u < RPL; ++u)
+          expand_row<DQ>(sQ + q * C::kQBytes, pre_q[q][u], q0 + q * BM + rbase + lane + 32 * u < N,
+                         rbase + lane + 32 * u, d);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars[Bar::qfull()]);
       for (int t = 0; t < T; ++t, ++g) {
         const int st = g % S;
-        const uint4 cb[2] = {nb[0], nb[1]};
+        uint4 cb[RPL];
+#pragma unroll
+        for (int u = 0; u < RPL; ++u) cb[u] = nb[u];
         // Sign rows of the next K block: this item's next block, or block 0 of the next item.
         {
           int64_t nbh = bh;
@@ -495,8 +513,8 @@ __global__ void __launch_bounds__(Cfg<DP, BK>::kThreads, 1)
           }
           const uint4* nrows = reinterpret_cast<const uint4*>(p.bits_k) + nbh * N;
 #pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int row = nt * BN + 64 * half + lane + 32 * u;
+          for (int u = 0; u < RPL; ++u) {
+            const int row = nt * BN + rbase + lane + 32 * u;
             nb[u] = (any && row < N) ? __ldg(nrows + row) : zero4;
           }
         }
@@ -505,8 +523,8 @@ __global__ void __launch_bounds__(Cfg<DP, BK>::kThreads, 1)
           break;
         }
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int r = 64 * half + lane + 32 * u;
+        for (int u = 0; u < RPL; ++u) {
+          const int r = rbase + lane + 32 * u;
           expand_row<DQ>(sK + st * C::kKBytes, cb[u], t * BN + r < N, r, d);
         }
         fence_proxy_async_smem();
@@ -514,8 +532,8 @@ __global__ void __launch_bounds__(Cfg<DP, BK>::kThreads, 1)
         if (lane == 0) mbar_arrive(&bars[Bar::kvfull(st)]);
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp < 4) {
+    // ------------------------------------------------------------ MMA issuer(s)
     // In order over the blocks j (counted across items): P.V(j) once group j % 2 has written
     // P(j) and the fold of block j - 1 has read the accumulator; then QK(j + 2) into the S buffer
     // that P(j) occupied (issue order keeps P read before S is rewritten). QK(0) and QK(1) first.
@@ -542,6 +560,45 @@ __global__ void __launch_bounds__(Cfg<DP, BK>::kThreads, 1)
         if (t == T - 1) tc_commit(&bars[Bar::qempty()]);  // the item's Q tile is free
         return true;
       };
+      if constexpr (C::kTilePP) {
+        // Two tiles, one S buffer and one accumulator each: P.V(q, n) once tile q's softmax has
+        // written P(n) (it folds block n - 1 out of the accumulator before that), then QK(q, n + 1)
+        // into the same S buffer (issue order keeps P read before S is rewritten). Tile 0's next
+        // QK is issued before tile 1's P.V wait, so neither tile's softmax waits on the other's.
+        auto qk_tile = [&](int q, int n) -> bool {
+          const int t = n % T;
+          if (q == 0) {
+            if (t == 0 && !wait_bounded(&bars[Bar::qfull()], (n / T) & 1, abort_flag)) return false;
+            if (!wait_bounded(&bars[Bar::kvfull(n % S)], (n / S) & 1, abort_flag)) return false;
+            tc_fence_after();
+          }
+          const uint32_t qb = smem_u32(sQ + q * C::kQBytes), kb = smem_u32(sK + (n % S) * C::kKBytes);
+#pragma unroll
+          for (int kk = 0; kk < DQ / 32; ++kk)
+            mma_f8f6f4_ss(tmem + C::tS(q, 0), smem_desc(qb + kk * 4096, 2048, 128),
+                          smem_desc(kb + kk * 4096, 2048, 128), idesc_qk, kk > 0 ? 1u : 0u);
+          tc_commit(&bars[Bar::sfull(q, 0)]);
+          if (q == 1 && t == T - 1) tc_commit(&bars[Bar::qempty()]);  // both tiles of the item read Q
+          return true;
+        };
+        auto pv_tile = [&](int q, int n) -> bool {
+          if (!wait_bounded(&bars[Bar::pfull(q)], n & 1, abort_flag)) return false;
+          tc_fence_after();
+          const uint32_t vbase = smem_u32(sV + (n % S) * C::kVBytes);
+#pragma unroll
+          for (int kk = 0; kk < BN / 32; ++kk)
+            mma_i8_ts(tmem + C::tAcc(q), tmem + C::tS(q, 0) + 8 * kk, smem_desc(vbase + 512 * kk, 128, 2048),
+                      idesc_pv, kk > 0 ? 1u : 0u);
+          tc_commit(&bars[Bar::pvdone(q)]);
+          if (q == 1) tc_commit(&bars[Bar::kvempty(n % S)]);  // the last reader of stage n
+          return true;
+        };
+        bool ok = nblocks == 0 || (qk_tile(0, 0) && qk_tile(1, 0));
+        for (int n = 0; n < nblocks && ok; ++n) {
+          const bool more = n + 1 < nblocks;
+          ok = pv_tile(0, n) && (!more || qk_tile(0, n + 1)) && pv_tile(1, n) && (!more || qk_tile(1, n + 1));
+        }
+      } else {
       bool ok = nblocks == 0 || qk(0);
       if (ok && nblocks > 1) ok = qk(1);
       for (int j = 0; j < nblocks && ok; ++j) {
@@ -556,6 +613,7 @@ __global__ void __launch_bounds__(Cfg<DP, BK>::kThreads, 1)
         tc_commit(&bars[Bar::pvdone(j & 1)]);
         tc_commit(&bars[Bar::kvempty(j % S)]);
         if (j + 2 < nblocks && !qk(j + 2)) break;
+      }
       }
       // Every MMA this thread issued has completed before tensor memory is released.
       tc_commit(&bars[Bar::drain()]);
@@ -578,14 +636,15 @@ __global__ void __launch_bounds__(Cfg<DP, BK>::kThreads, 1)
     //     P.V(j); P.V(j + 1) waits for it (one accumulator), so the folds, and every update of
     //     F', L' and m_ref, run in block order.
     const int grp = (warp - 4) >> 2, w4 = warp & 3;
+    const int qt = C::kTilePP ? grp : 0;  // this group's query tile
     const int r = w4 * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(w4 * 32) << 16;
-    const uint32_t aAcc = tmem + lane_base + C::tAcc(0);
-    const uint32_t aF = tmem + lane_base + C::tF(0);
+    const uint32_t aAcc = tmem + lane_base + C::tAcc(qt);
+    const uint32_t aF = tmem + lane_base + C::tF(qt);
     float* s_m = reinterpret_cast<float*>(smem + C::offX);  // [2][BM] m_j by block parity
-    // [BM] (L', m_ref) of each row, stored as one 8-byte pair so that a reader outside the fold
-    // chain sees a consistent pair.
-    float2* s_Lm = reinterpret_cast<float2*>(s_m + 2 * BM);
+    // [tile][BM] (L', m_ref) of each row, stored as one 8-byte pair so that a reader outside the
+    // fold chain sees a consistent pair.
+    float2* s_Lm = reinterpret_cast<float2*>(s_m + 2 * BM) + qt * BM;
     uint64_t* mch = &bars[Bar::mchain(w4)];
     // Share of the error bar one changed code may take in a row that is not checked.
     constexpr float kCheckTau = 2.0e-4f;
@@ -596,9 +655,9 @@ __global__ void __launch_bounds__(Cfg<DP, BK>::kThreads, 1)
     for (int it = 0; it < n_items && alive; ++it, n0 += T) {
       int64_t bh;
       int q0;
-      item_at(by_head, it, p.H, nqb, BM, bh, q0);
+      item_at(by_head, it, p.H, nqb, BM * NQ, bh, q0);
       const int64_t b = bh / p.H, h = bh - b * p.H;
-      const int i = q0 + r;
+      const int i = q0 + qt * BM + r;
       const bool row_ok = i < N;
       const int ic = row_ok ? i : N - 1;  // rows past N read the bias of row N-1 (never stored)
       if (it == 0) {
@@ -646,20 +705,90 @@ __global__ void __launch_bounds__(Cfg<DP, BK>::kThreads, 1)
       // below must not depend on when the other group's fold lands, or results would vary
       // from run to run); L' = 0 before the group's first fold of the item.
       float own_L = 0.0f, own_mref = 0.0f;
+      // Tile ping-pong: the running maximum, and the sum and maximum of the block awaiting its
+      // fold, in registers.
+      float m_run = -CUDART_INF_F, lt_prev = 0.0f;
 
-      for (int t = grp ^ (n0 & 1); t < T && alive; t += 2) {
+      // The fold of block tb (item-relative; running maximum m_b, sum of P~ lt_b):
+      // F' += acc e, L' += lt_b e with e = exp(m_b - m_ref) (the item's first block sets F' = acc,
+      // L' = lt_b, m_ref = m_b; e beyond 2^64 moves m_ref up to m_b, rescaling F' and L').
+      auto fold_block = [&](int tb, float m_b, float lt_b) {
+        float e = 1.0f, ratio = 1.0f;
+        float mref = m_b, Lp = 0.0f;
+        if (tb > 0) {
+          const float2 lm = s_Lm[r];
+          Lp = lm.x;
+          mref = lm.y;
+          e = ex2_approx((m_b - mref) * kLog2e);
+          if (e > 1.8446744e19f) {
+            ratio = 1.0f / e;
+            e = 1.0f;
+            mref = m_b;
+          }
+        }
+        const bool rescale = __any_sync(0xffffffffu, ratio != 1.0f);
+        auto fold = [&](auto first) {
+          constexpr bool FIRST = decltype(first)::value;
+#pragma unroll 1
+          for (int c0 = 0; c0 < DP; c0 += 32) {
+            constexpr int G = 32;
+            uint32_t a[G], f[G];
+            if (c0 + G <= DP) {
+              tmem_ld_cols<G>(aAcc + c0, a);
+              if (!FIRST) tmem_ld_cols<G>(aF + c0, f);
+            } else {
+              tmem_ld_cols<16>(aAcc + c0, a);
+              if (!FIRST) tmem_ld_cols<16>(aF + c0, f);
+            }
+            tmem_ld_wait();
+            reg_fence_cols<G>(a);
+            if (!FIRST) reg_fence_cols<G>(f);
+            const float2 e2 = make_float2(e, e), rt2 = make_float2(ratio, ratio);
+#pragma unroll
+            for (int k = 0; k < G; k += 2) {
+              const float2 a2 = __fadd2_rn(
+                  make_float2(__uint_as_float(a[k] + kMagicBits), __uint_as_float(a[k + 1] + kMagicBits)),
+                  make_float2(-kMagic, -kMagic));
+              float2 f2;
+              if (FIRST) {
+                f2 = a2;
+              } else {
+                float2 fo = make_float2(__uint_as_float(f[k]), __uint_as_float(f[k + 1]));
+                if (rescale) fo = __fmul2_rn(fo, rt2);
+                f2 = __ffma2_rn(a2, e2, fo);
+              }
+              f[k] = __float_as_uint(f2.x);
+              f[k + 1] = __float_as_uint(f2.y);
+            }
+            if (c0 + G <= DP)
+              tmem_st_cols<G>(aF + c0, f);
+            else
+              tmem_st_cols<16>(aF + c0, f);
+          }
+        };
+        if (tb == 0)
+          fold(std::true_type{});
+        else
+          fold(std::false_type{});
+        own_L = (tb == 0) ? lt_b : __fmaf_rn(lt_b, e, Lp * ratio);
+        own_mref = mref;
+        s_Lm[r] = make_float2(own_L, own_mref);
+      };
+
+      for (int t = C::kTilePP ? 0 : (grp ^ (n0 & 1)); t < T && alive; t += C::kTilePP ? 1 : 2) {
         const int n = n0 + t;
         const int st = n % S;
         const int j0 = t * BN;
         const int nk = min(BN, N - j0);  // valid keys of this block
-        const uint32_t aS = tmem + lane_base + C::tS(0, n & 1);
+        const uint32_t aS = tmem + lane_base + (C::kTilePP ? C::tS(qt, 0) : C::tS(0, n & 1));
         if constexpr (BK == kRelWindow || is_relpos_general(BK)) {
           if (!wait_warp(&bars[Bar::kvfull(st)], (n / S) & 1, abort_flag)) {
             alive = false;
             break;
           }
         }
-        if (!wait_warp(&bars[Bar::sfull(0, n & 1)], (n >> 1) & 1, abort_flag)) {
+        if (!wait_warp(&bars[C::kTilePP ? Bar::sfull(qt, 0) : Bar::sfull(0, n & 1)],
+                       C::kTilePP ? (n & 1) : ((n >> 1) & 1), abort_flag)) {
           alive = false;
           break;
         }
@@ -696,8 +825,8 @@ __global__ void __launch_bounds__(Cfg<DP, BK>::kThreads, 1)
             if constexpr (BK == kRelWindow) {
               // Every chunk lies in one grid row (grid width a multiple of 32, N = grid size), so
               // its 32 biases are a descending run of the window. Chunks past N are masked.
-              const int kc = jc < N ? swink[st * 4 + c] : A_i - 31;
-              wrow = swin + st * kWinFloats + (A_i - kc);
+              const int kc = jc < N ? swink[(st * NQ + qt) * 4 + c] : A_i - 31;
+              wrow = swin + (st * NQ + qt) * kWinFloats + (A_i - kc);
             }
 #pragma unroll
             for (int g8 = 0; g8 < 4; ++g8) {
@@ -769,19 +898,38 @@ __global__ void __launch_bounds__(Cfg<DP, BK>::kThreads, 1)
         const float bmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
         tmem_st_wait();  // s is in S before pass 2 reads it back
 
-        // ---- the running maximum: m_{n-1} from the other group (block n - 1), then m_n out
+        // ---- the running maximum: tile ping-pong, in a register; block ping-pong, m_{n-1} from
+        // the other group (block n - 1), then m_n out
         float m_prev = -CUDART_INF_F;
-        if (n > 0) {
-          if (!wait_warp(mch, (n - 1) & 1, abort_flag)) {
+        if constexpr (C::kTilePP) {
+          m_prev = (t == 0) ? -CUDART_INF_F : m_run;
+        } else {
+          if (n > 0) {
+            if (!wait_warp(mch, (n - 1) & 1, abort_flag)) {
+              alive = false;
+              break;
+            }
+            if (t > 0) m_prev = s_m[((n - 1) & 1) * BM + r];
+          }
+        }
+        const float m_new = fmaxf(m_prev, bmax);
+        if constexpr (!C::kTilePP) {
+          s_m[(n & 1) * BM + r] = m_new;
+          __syncwarp();
+          if (lane == 0) mbar_arrive(mch);
+        } else if (t > 0) {
+          // Fold block n - 1 (its P.V completed before QK(n), which this block's S came from).
+          if (!wait_warp(&bars[Bar::pvdone(qt)], (n - 1) & 1, abort_flag)) {
             alive = false;
             break;
           }
-          if (t > 0) m_prev = s_m[((n - 1) & 1) * BM + r];
+          tc_fence_after();
+          fold_block(t - 1, m_prev, lt_prev);
+          tmem_st_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars[Bar::folddone(qt)]);
         }
-        const float m_new = fmaxf(m_prev, bmax);
-        s_m[(n & 1) * BM + r] = m_new;
-        __syncwarp();
-        if (lane == 0) mbar_arrive(mch);
         // Rows whose softmax sum so far is small get the exact near-tie check. The sum is taken
         // as of this group's own last fold (an underestimate of the row's true sum).
         const float l_so_far = own_L > 0.0f ? own_L * ex2_approx((own_mref - m_new) * kLog2e) : 0.0f;
@@ -882,6 +1030,11 @@ __global__ void __launch_bounds__(Cfg<DP, BK>::kThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars[Bar::pfull(grp)]);
+        if constexpr (C::kTilePP) {
+          m_run = m_new;
+          lt_prev = lt;
+          continue;
+        }
 
         // ---- fold block n: F' += acc e_n, L' += l_n e_n (after P.V(n), which followed the fold
         // of block n - 1; at an item's first block also after both groups' previous epilogue)
@@ -898,68 +1051,7 @@ __global__ void __launch_bounds__(Cfg<DP, BK>::kThreads, 1)
           break;
         }
         tc_fence_after();
-        {
-          float e = 1.0f, ratio = 1.0f;
-          float mref = m_new, Lp = 0.0f;
-          if (t > 0) {
-            const float2 lm = s_Lm[r];
-            Lp = lm.x;
-            mref = lm.y;
-            e = ex2_approx((m_new - mref) * kLog2e);
-            if (e > 1.8446744e19f) {  // 2^64: move the reference up to m_n, rescaling F' and L'
-              ratio = 1.0f / e;
-              e = 1.0f;
-              mref = m_new;
-            }
-          }
-          const bool rescale = __any_sync(0xffffffffu, ratio != 1.0f);
-          auto fold = [&](auto first) {
-            constexpr bool FIRST = decltype(first)::value;  // the item's first block: F' = acc
-#pragma unroll 1
-            for (int c0 = 0; c0 < DP; c0 += 32) {
-              constexpr int G = 32;
-              uint32_t a[G], f[G];
-              if (c0 + G <= DP) {
-                tmem_ld_cols<G>(aAcc + c0, a);
-                if (!FIRST) tmem_ld_cols<G>(aF + c0, f);
-              } else {
-                tmem_ld_cols<16>(aAcc + c0, a);
-                if (!FIRST) tmem_ld_cols<16>(aF + c0, f);
-              }
-              tmem_ld_wait();
-              reg_fence_cols<G>(a);
-              if (!FIRST) reg_fence_cols<G>(f);
-              const float2 e2 = make_float2(e, e), rt2 = make_float2(ratio, ratio);
-#pragma unroll
-              for (int k = 0; k < G; k += 2) {
-                const float2 a2 = __fadd2_rn(
-                    make_float2(__uint_as_float(a[k] + kMagicBits), __uint_as_float(a[k + 1] + kMagicBits)),
-                    make_float2(-kMagic, -kMagic));
-                float2 f2;
-                if (FIRST) {
-                  f2 = a2;
-                } else {
-                  float2 fo = make_float2(__uint_as_float(f[k]), __uint_as_float(f[k + 1]));
-                  if (rescale) fo = __fmul2_rn(fo, rt2);
-                  f2 = __ffma2_rn(a2, e2, fo);
-                }
-                f[k] = __float_as_uint(f2.x);
-                f[k + 1] = __float_as_uint(f2.y);
-              }
-              if (c0 + G <= DP)
-                tmem_st_cols<G>(aF + c0, f);
-              else
-                tmem_st_cols<16>(aF + c0, f);
-            }
-          };
-          if (t == 0)
-            fold(std::true_type{});
-          else
-            fold(std::false_type{});
-          own_L = (t == 0) ? lt : __fmaf_rn(lt, e, Lp * ratio);
-          own_mref = mref;
-          s_Lm[r] = make_float2(own_L, own_mref);
-        }
+        fold_block(t, m_new, lt);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
@@ -972,12 +1064,24 @@ __global__ void __launch_bounds__(Cfg<DP, BK>::kThreads, 1)
       if (it + 1 < n_items) {
         int64_t nbh;
         int nq0;
-        item_at(by_head, it + 1, p.H, nqb, BM, nbh, nq0);
+        item_at(by_head, it + 1, p.H, nqb, BM * NQ, nbh, nq0);
         mu_q_next = p.mu_q[nbh];
         mu_k_next = p.mu_k[nbh];
       }
       const int nl = n0 + T - 1;  // the item's last block
-      if (!wait_warp(&bars[Bar::folddone(nl & 1)], (nl >> 1) & 1, abort_flag)) {
+      if constexpr (C::kTilePP) {
+        // The item's last block: its P.V, then its fold.
+        if (!wait_warp(&bars[Bar::pvdone(qt)], nl & 1, abort_flag)) {
+          alive = false;
+          break;
+        }
+        tc_fence_after();
+        fold_block(T - 1, m_run, lt_prev);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[Bar::folddone(qt)]);
+      } else if (!wait_warp(&bars[Bar::folddone(nl & 1)], (nl >> 1) & 1, abort_flag)) {
         alive = false;
         break;
       }
@@ -985,9 +1089,11 @@ __global__ void __launch_bounds__(Cfg<DP, BK>::kThreads, 1)
       const float inv_l = 1.0f / (255.0f * s_Lm[r].x);
       const int esz = (p.o_dt == BA_F32) ? 4 : 2;
       const bool vec = ((d * esz) & 15) == 0;
+      // Block ping-pong: each group writes half of the row's channels; tile ping-pong: all.
+      constexpr int kChan = C::kTilePP ? DP : DH;
 #pragma unroll 1
-      for (int g0 = 0; g0 < DH; g0 += 8) {
-        const int c0 = grp * DH + g0;  // eight channels at a time of this group's DH
+      for (int g0 = 0; g0 < kChan; g0 += 8) {
+        const int c0 = (C::kTilePP ? 0 : grp * DH) + g0;  // eight channels at a time
         uint32_t f[8];
         tmem_ld_cols<8>(aF + c0, f);
         tmem_ld_wait();
@@ -1024,9 +1130,11 @@ __global__ void __launch_bounds__(Cfg<DP, BK>::kThreads, 1)
             if (c0 + k < d) store_out(p.o, (bh * N + i) * d + c0 + k, val[k], p.o_dt);
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[Bar::epidone()]);
+      if constexpr (!C::kTilePP) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[Bar::epidone()]);
+      }
     }
   }
 
