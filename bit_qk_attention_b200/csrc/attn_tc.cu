@@ -40,6 +40,7 @@
 #include <math_constants.h>
 
 #include <algorithm>
+#include <cmath>
 #include <type_traits>
 #include <mutex>
 
@@ -265,18 +266,45 @@ __device__ __forceinline__ void reg_fence_cols(uint32_t* r) {
   }
 }
 
-// The 8-bit code of one logit taken exactly as the definition states: P~ = exp(s - m) in double
-// rounded to fp32, 255 P~ rounded to fp32, then to the nearest integer (ties to even).
-__device__ __forceinline__ uint32_t exact_code(float s, float m) {
-  const float pe = static_cast<float>(exp(static_cast<double>(s) - static_cast<double>(m)));
-  const int c = __float2int_rn(__fmul_rn(255.0f, pe));
-  return static_cast<uint32_t>(min(255, max(0, c)));
+// Exact 8-bit codes at a rounding tie. The definition's code of a logit s against the running
+// max m is rne(fl32(255 fl32(exp(d)))), capped at 255, with d = (double)s - (double)m. It is a
+// non-decreasing function of d, so code(d) >= k + 1 exactly when d >= thr[k], the least double
+// whose code exceeds k. The host computes the 255 thresholds once, by bisection over doubles.
+struct TieTable {
+  double thr[256];
+};
+
+// Check mode rounds each 255 P~ twice, scaled by (1 - eps) and by (1 + eps). The two codes
+// differ only where 255 P~ lies within a relative eps of a rounding tie. eps bounds the
+// relative error of the fast path's P~ against fl32(exp(d)): the rounding of s - m and of its
+// product with log2 e (|t| <= 9 for a nonzero code), the hardware 2^t and the definition's two
+// fp32 roundings add up to about 1.2e-6.
+constexpr float kTieEps = 4.0e-6f;
+constexpr float kC255Lo = 255.0f * (1.0f - kTieEps);
+constexpr float kC255Hi = 255.0f * (1.0f + kTieEps);
+
+// One packed word of four codes: `hi` from the (1 + eps) rounding (the code wherever the two
+// agree), `lo` from the (1 - eps) one. Where they differ the exact code is lo or lo + 1, and
+// the key's d against thr[lo] decides.
+__device__ __forceinline__ uint32_t settle_ties(uint32_t hi, uint32_t lo, const uint32_t* xs, float m,
+                                                const TieTable& tt) {
+  uint32_t out = hi;
+#pragma unroll
+  for (int b = 0; b < 4; ++b) {
+    const uint32_t cl = (lo >> (8 * b)) & 0xFFu;
+    if (cl != ((hi >> (8 * b)) & 0xFFu)) {
+      const double dd = static_cast<double>(__uint_as_float(xs[b])) - static_cast<double>(m);
+      const uint32_t code = cl + (dd >= tt.thr[cl] ? 1u : 0u);
+      out = (out & ~(0xFFu << (8 * b))) | (code << (8 * b));
+    }
+  }
+  return out;
 }
 
 template <int DP, int BK>
 __global__ void __launch_bounds__(Cfg<DP, BK>::kThreads, 1)
     attn_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmap_v, int tab_mode, int tsize,
-                   int kmax, int win_stride) {
+                   int kmax, int win_stride, const __grid_constant__ TieTable tie) {
   using C = Cfg<DP, BK>;
   constexpr int NQ = C::NQ, SB = C::SB, DQ = C::DQ, DH = C::DH, S = C::kStages;
   using Bar = Bars<C>;
@@ -648,7 +676,6 @@ __global__ void __launch_bounds__(Cfg<DP, BK>::kThreads, 1)
     uint64_t* mch = &bars[Bar::mchain(w4)];
     // Share of the error bar one changed code may take in a row that is not checked.
     constexpr float kCheckTau = 2.0e-4f;
-    constexpr float kTieBand = 0.5f - 2.5e-4f;
     bool alive = true;
     float mu_q_next = 0.0f, mu_k_next = 0.0f;  // mu of the item about to start (loaded one item ahead)
     int n0 = 0;  // index, counted across items, of the item's first key block
@@ -936,11 +963,14 @@ __global__ void __launch_bounds__(Cfg<DP, BK>::kThreads, 1)
         const bool check = p.p_check_all || __any_sync(0xffffffffu, l_so_far + 1.0f < l_check);
 
         // ---- pass 2: P~ = 2^((s - m) log2 e), row sum, 8-bit codes (masked keys: s = -inf,
-        // P~ = 0) per 32-key chunk, near-tie codes of each 16-key group settled in place; the
-        // codes go to columns 8c .. 8c + 7 of the S buffer (keys 0..31 of S, read already).
+        // P~ = 0) per 32-key chunk; in check mode each 4-key word's near-tie codes are settled in
+        // place. The codes go to columns 8c .. 8c + 7 of the S buffer (keys 0..31 of S, read
+        // already).
         const float2 negm2 = make_float2(-m_new, -m_new);
         const float2 log2e2 = make_float2(kLog2e, kLog2e);
         const float2 c255 = make_float2(255.0f, 255.0f);
+        const float2 c255lo = make_float2(kC255Lo, kC255Lo);
+        const float2 c255hi = make_float2(kC255Hi, kC255Hi);
         const float2 magic2 = make_float2(kMagic, kMagic);
         float2 lt2[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
         auto pass2 = [&](auto checked) {
@@ -962,54 +992,31 @@ __global__ void __launch_bounds__(Cfg<DP, BK>::kThreads, 1)
             if (c + 1 < BN / 32) tmem_ld_cols<32>(aS + 32 * (c + 1), xn);
             uint32_t pk[8];
 #pragma unroll
-            for (int g4 = 0; g4 < 2; ++g4) {
-              float rmx = 0.0f;
+            for (int w = 0; w < 8; ++w) {
+              uint32_t y[4], yl[4];
 #pragma unroll
-              for (int w = 4 * g4; w < 4 * g4 + 4; ++w) {
-                uint32_t y[4];
-#pragma unroll
-                for (int e2 = 0; e2 < 2; ++e2) {
-                  const int k = 4 * w + 2 * e2;
-                  // s - m first (exact near the maximum), then the scale to base 2.
-                  const float2 t2 = __fmul2_rn(
-                      __fadd2_rn(make_float2(__uint_as_float(x[k]), __uint_as_float(x[k + 1])), negm2), log2e2);
-                  const float2 p2 = make_float2(ex2_approx(t2.x), ex2_approx(t2.y));
-                  lt2[e2] = __fadd2_rn(lt2[e2], p2);
-                  // 255 P~ + 1.5 * 2^23: one rounding to the nearest integer (ties to even); the
-                  // integer sits in the low byte of the result (P~ <= 1).
-                  const float2 y2 = __ffma2_rn(p2, c255, magic2);
-                  y[2 * e2] = __float_as_uint(y2.x);
-                  y[2 * e2 + 1] = __float_as_uint(y2.y);
-                  if (CHECK) {
-                    // Distance of 255 P~ from the code it rounded to; near 1/2 the fast
-                    // exponential's error can decide the code.
-                    const float2 r2 = __ffma2_rn(p2, c255, __fadd2_rn(magic2, make_float2(-y2.x, -y2.y)));
-                    rmx = fmax3(rmx, fabsf(r2.x), fabsf(r2.y));
-                  }
+              for (int e2 = 0; e2 < 2; ++e2) {
+                const int k = 4 * w + 2 * e2;
+                // s - m first (exact near the maximum), then the scale to base 2.
+                const float2 t2 = __fmul2_rn(
+                    __fadd2_rn(make_float2(__uint_as_float(x[k]), __uint_as_float(x[k + 1])), negm2), log2e2);
+                const float2 p2 = make_float2(ex2_approx(t2.x), ex2_approx(t2.y));
+                lt2[e2] = __fadd2_rn(lt2[e2], p2);
+                // 255 P~ + 1.5 * 2^23: one rounding to the nearest integer (ties to even); the
+                // integer sits in the low byte of the result (P~ <= 1).
+                const float2 y2 = __ffma2_rn(p2, CHECK ? c255hi : c255, magic2);
+                y[2 * e2] = __float_as_uint(y2.x);
+                y[2 * e2 + 1] = __float_as_uint(y2.y);
+                if (CHECK) {
+                  const float2 z2 = __ffma2_rn(p2, c255lo, magic2);
+                  yl[2 * e2] = __float_as_uint(z2.x);
+                  yl[2 * e2 + 1] = __float_as_uint(z2.y);
                 }
-                pk[w] = __byte_perm(__byte_perm(y[0], y[1], 0x0040), __byte_perm(y[2], y[3], 0x0040), 0x5410);
               }
-              if (CHECK && rmx > kTieBand) {
-                // Rare: settle this group's near-tie codes one key at a time (a rolled loop over a
-                // small local copy, so the double-precision exponential appears once).
-                float sg[16];
-                uint32_t pw[4];
-#pragma unroll
-                for (int k = 0; k < 16; ++k) sg[k] = __uint_as_float(x[16 * g4 + k]);
-#pragma unroll
-                for (int k = 0; k < 4; ++k) pw[k] = pk[4 * g4 + k];
-#pragma unroll 1
-                for (int k = 0; k < 16; ++k) {
-                  const float pk1 = ex2_approx(__fmul_rn(__fadd_rn(sg[k], -m_new), kLog2e));
-                  const float rk = __fmaf_rn(pk1, 255.0f, __fadd_rn(kMagic, -__fmaf_rn(pk1, 255.0f, kMagic)));
-                  if (fabsf(rk) > kTieBand) {
-                    const uint32_t code = exact_code(sg[k], m_new);
-                    const uint32_t sh = 8u * static_cast<uint32_t>(k & 3);
-                    pw[k >> 2] = (pw[k >> 2] & ~(0xFFu << sh)) | (code << sh);
-                  }
-                }
-#pragma unroll
-                for (int k = 0; k < 4; ++k) pk[4 * g4 + k] = pw[k];
+              pk[w] = __byte_perm(__byte_perm(y[0], y[1], 0x0040), __byte_perm(y[2], y[3], 0x0040), 0x5410);
+              if (CHECK) {
+                const uint32_t pl = __byte_perm(__byte_perm(yl[0], yl[1], 0x0040), __byte_perm(yl[2], yl[3], 0x0040), 0x5410);
+                if (pl != pk[w]) pk[w] = settle_ties(pk[w], pl, x + 4 * w, m_new, tie);
               }
             }
             tmem_st_cols<8>(aS + 8 * c, pk);
@@ -1191,6 +1198,35 @@ int window_stride(const AttnParams& p) {
   return static_cast<int64_t>(ndy) * ws <= kWinFloats ? ws : 0;
 }
 
+// The thresholds of the exact P codes (TieTable): thr[k] is the least double d with
+// code(d) >= k + 1, code(d) = min(255, rne(fl32(255 fl32(exp(d))))), found by bisection between
+// adjacent doubles (code(-1000) = 0, code(0) = 255). Computed once per process.
+const TieTable& tie_table() {
+  static const TieTable table = [] {
+    TieTable t{};
+    auto code = [](double d) {
+      const float pe = static_cast<float>(std::exp(d));
+      const float c = std::nearbyint(255.0f * pe);
+      return c > 255.0f ? 255 : static_cast<int>(c);
+    };
+    for (int k = 0; k < 255; ++k) {
+      double lo = -1000.0, hi = 0.0;
+      for (;;) {
+        const double mid = lo + 0.5 * (hi - lo);
+        if (!(mid > lo && mid < hi)) break;
+        if (code(mid) >= k + 1)
+          hi = mid;
+        else
+          lo = mid;
+      }
+      t.thr[k] = hi;
+    }
+    t.thr[255] = HUGE_VAL;  // a settled key's lower code is at most 254
+    return t;
+  }();
+  return table;
+}
+
 template <int DP, int BK>
 cudaError_t launch_cfg(const AttnParams& p, const CUtensorMap& tm, cudaStream_t s) {
   using C = Cfg<DP, BK>;
@@ -1242,7 +1278,7 @@ cudaError_t launch_cfg(const AttnParams& p, const CUtensorMap& tm, cudaStream_t 
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kernel, p, tm, tab_mode, tsize, kmax, wst);
+  return cudaLaunchKernelEx(&cfg, kernel, p, tm, tab_mode, tsize, kmax, wst, tie_table());
 }
 
 template <int DP>
