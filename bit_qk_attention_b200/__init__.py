@@ -50,6 +50,7 @@ SIGNATURES = {
     "ba_sign_words": (_I, [_I]),
     "ba_v_row_bytes": (_I, [_I]),
     "ba_kv_block": (_I, []),
+    "ba_p_code_threshold": (ctypes.c_double, [_I]),
     "ba_prep_fused": (_I, [_I, _I, _I, _I]),
     "ba_pack_workspace_bytes": (_SZ, [_I, _I, _I, _I]),
     "ba_quant_workspace_bytes": (_SZ, [_I, _I, _I, _I]),
@@ -166,6 +167,11 @@ def v_row_bytes(d: int) -> int:
 
 def kv_block() -> int:
     return lib().ba_kv_block()
+
+
+def p_code_threshold(k: int) -> float:
+    """The least d = s - m (double) whose 8-bit P code exceeds k (0 <= k <= 254), else NaN."""
+    return lib().ba_p_code_threshold(int(k))
 
 
 def prep_fused(B: int, H: int, N: int, d: int) -> bool:

@@ -226,6 +226,8 @@ int ba_v_row_bytes(int d) { return (d >= 1 && d <= 128) ? v_row_bytes(d) : 0; }
 
 int ba_kv_block(void) { return kKvBlock; }
 
+double ba_p_code_threshold(int k) { return p_code_threshold(k); }
+
 int ba_prep_fused(int B, int H, int N, int d) {
   if (check_dims(B, H, N, d) != BA_OK || empty(B, H, N)) return 0;
   return use_slice_prep(dims(B, H, N, d)) ? 1 : 0;

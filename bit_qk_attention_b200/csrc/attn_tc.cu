@@ -1332,6 +1332,8 @@ cudaError_t launch_dp(const AttnParams& p, const CUtensorMap& tm, cudaStream_t s
 
 }  // namespace
 
+double p_code_threshold(int k) { return (k >= 0 && k < 255) ? tie_table().thr[k] : std::nan(""); }
+
 bool attn_tc_supported(const AttnParams& p) {
   return p.dp >= 16 && p.dp <= 128 && (p.dp % 16) == 0 && p.N >= 1 && encode_fn() != nullptr;
 }

@@ -79,6 +79,7 @@ cudaError_t launch_quant(const QuantParams& p, int dt, cudaStream_t s);
 // Fused attention on packed operands.
 cudaError_t launch_attn_simt(const AttnParams& p, cudaStream_t s);
 bool attn_tc_supported(const AttnParams& p);
+double p_code_threshold(int k);  // the exact-code threshold table of the tcgen05 kernel
 cudaError_t launch_attn_tc(const AttnParams& p, cudaStream_t s);
 
 // Device status word of the kernels with bounded waits.

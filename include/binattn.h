@@ -79,6 +79,14 @@ int ba_v_row_bytes(int d);
 int ba_kv_block(void);
 
 /*
+ * The exact-code thresholds the tcgen05 kernel uses near a rounding tie: for 0 <= k <= 254, the
+ * least double d whose code min(255, rne(fl32(255 * fl32(exp(d))))) exceeds k (the code of a
+ * logit s against the running max m, with d = (double)s - (double)m; gist.science/zh 2.2(3)).
+ * NaN for any other k. Host-side; computed once per process.
+ */
+double ba_p_code_threshold(int k);
+
+/*
  * Preparation path ba_attention_fwd takes for this shape: 1 = one launch (one CTA per (b, h)
  * slice and tensor writes the sign bits and mu of q and k and the scales and int8 rows of v;
  * taken for many short slices with d a multiple of 8 and d >= 32), 0 = three launches

@@ -67,6 +67,30 @@ def test_host_queries(L):
         assert L.ba_status_string(s).startswith(b"BA_")
 
 
+def test_p_code_thresholds(L):
+    """The tcgen05 kernel's exact-code thresholds against the definition's P code of
+    d = s - m, written out here: code(d) = min(255, rne(fl32(255 * fl32(exp(d))))). Each
+    threshold is the least double whose code exceeds k: its code is at least k + 1, and the next
+    double below it has a code of at most k."""
+    import math
+    import numpy as np
+
+    def code(d):
+        p = np.float32(math.exp(d))
+        return int(min(np.rint(np.float32(255.0) * p), 255.0))
+
+    prev = -math.inf
+    for k in range(255):
+        t = L.ba_p_code_threshold(k)
+        assert prev < t < 0.0
+        assert code(t) >= k + 1
+        assert code(math.nextafter(t, -math.inf)) <= k
+        # the real boundary 255 exp(d) = k + 1/2, moved only by the two fp32 roundings
+        assert abs(t - math.log((k + 0.5) / 255.0)) < 1e-6
+        prev = t
+    assert math.isnan(L.ba_p_code_threshold(255)) and math.isnan(L.ba_p_code_threshold(-1))
+
+
 def test_noalloc_limit_matches_header():
     import bit_qk_attention_b200 as ba
     text = open(HEADER).read()
