@@ -287,6 +287,7 @@ ba_status ba_quant_v(const void* v, ba_dtype dt, int B, int H, int N, int d, int
   qp.v_scale = v_scale;
   qp.vq = vq;
   qp.npack = 0;
+  qp.tpc = quant_tokens_per_cta(g);
   return cuda_status(launch_quant(qp, dt, s));
 }
 
@@ -383,6 +384,7 @@ ba_status forward(const void* q, const void* k, const void* v, ba_dtype dt, int 
     qp.v_scale = at<float>(ws, L.v_scale);
     qp.vq = at<int8_t>(ws, L.vq);
     qp.npack = 2;
+    qp.tpc = quant_tokens_per_cta(g);
     qp.part_mu[0] = at<double>(ws, L.part_mu_q);
     qp.part_mu[1] = at<double>(ws, L.part_mu_k);
     qp.mu[0] = at<float>(ws, L.mu_q);

@@ -10,7 +10,7 @@ namespace binattn {
 
 constexpr int kJobPack = 0;  // sign bits + sum |x| per chunk
 constexpr int kJobAmax = 1;  // per-channel max |v| per group of chunks
-constexpr int kQuantTokens = 1024;  // tokens per CTA of the V quantiser
+constexpr int kQuantTokens = 1024;  // most tokens per CTA of the V quantiser
 
 struct PrepDims {
   int64_t BH;
@@ -39,10 +39,11 @@ struct FinalizeParams {
 };
 
 // V quantiser with the finalize folded in: each CTA reduces its slice's partial channel maxima
-// (npart rows of dp floats), then writes int8 rows for kQuantTokens tokens; a slice's first CTA
-// also writes the V scales and the mu of up to two packed tensors from their chunk sums.
+// (npart rows of dp floats), then writes int8 rows for tpc tokens; a slice's first CTA also
+// writes the V scales and the mu of up to two packed tensors from their chunk sums.
 struct QuantParams {
   PrepDims g;
+  int tpc;  // tokens per CTA (quant_tokens_per_cta)
   const void* v;
   const float* part_amax;  // [BH][npart][dp]
   int npart;
@@ -75,6 +76,7 @@ bool use_slice_prep(const PrepDims& g);
 int amax_parts(const PrepDims& g);  // partial channel-max rows per slice written by launch_prep
 cudaError_t launch_finalize(const FinalizeParams& p, cudaStream_t s);
 cudaError_t launch_quant(const QuantParams& p, int dt, cudaStream_t s);
+int quant_tokens_per_cta(const PrepDims& g);
 
 // Fused attention on packed operands.
 cudaError_t launch_attn_simt(const AttnParams& p, cudaStream_t s);

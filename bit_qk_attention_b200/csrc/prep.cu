@@ -6,7 +6,7 @@
 //                       sign bits + per-chunk sum |x| of q and k; one CTA per eight chunks of
 //                       v, their channel max |v|;
 //   prep_kernel       — d % 8 != 0: a CTA per (tensor, chunk), the same per-chunk partials;
-//   quant_kernel      — V -> int8 rows, 1024 tokens per CTA; each CTA reduces its slice's
+//   quant_kernel      — V -> int8 rows, 128-1024 tokens per CTA; each CTA reduces its slice's
 //                       channel-max partials to the inverse scales itself, and a slice's first
 //                       CTA writes mu of q and k and the V scales (no separate finalize launch);
 //   finalize_kernel   — mu = sum / (N d) per (b, h), for sign packing on its own.
@@ -141,14 +141,14 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(QuantParams p) {
   __shared__ float sinv[128];
   const PrepDims& g = p.g;
   const int d = g.d, dp = g.dp;
-  const int ngrp = (g.N + kQuantTokens - 1) / kQuantTokens;
+  const int ngrp = (g.N + p.tpc - 1) / p.tpc;
   // Last slice first: the streaming kernel before this one reads V in slice order, so the
   // slices it read last are the likeliest to be still in L2.
   const int64_t cta = static_cast<int64_t>(gridDim.x) - 1 - blockIdx.x;
   const int64_t bh = cta / ngrp;
   const int grp = static_cast<int>(cta - bh * ngrp);
-  const int tok0 = grp * kQuantTokens;
-  const int ntok = min(kQuantTokens, g.N - tok0);
+  const int tok0 = grp * p.tpc;
+  const int ntok = min(p.tpc, g.N - tok0);
   const bool vec = (d & 7) == 0;
   // Vector path: thread (rp, sub) writes the 8-byte piece sub of rows rp + rpp t; pieces at or
   // past d are the zero padding of the row.
@@ -675,11 +675,20 @@ cudaError_t launch_prep_slices(const SliceParams& p, int dt, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+// Tokens per quantiser CTA: 1024, halved (down to 128) while the grid would hold fewer than 512
+// CTAs, so that short slices still spread over every SM.
+int quant_tokens_per_cta(const PrepDims& g) {
+  int tpc = kQuantTokens;
+  while (tpc > kPrepTokens && g.BH * ceil_div(g.N, tpc) < 512) tpc /= 2;
+  return tpc;
+}
+
 // A programmatic dependent of the streaming kernel: its CTAs may be resident, with their first
 // V loads in flight, before that grid completes.
 cudaError_t launch_quant(const QuantParams& p, int dt, cudaStream_t s) {
+  if (p.tpc < 1) return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(static_cast<unsigned>(p.g.BH * ceil_div(p.g.N, kQuantTokens)));
+  cfg.gridDim = dim3(static_cast<unsigned>(p.g.BH * ceil_div(p.g.N, p.tpc)));
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = s;
