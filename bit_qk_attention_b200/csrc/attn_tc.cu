@@ -1107,24 +1107,37 @@ __global__ void __launch_bounds__(Cfg<DP, BK>::kThreads, 1)
         mu_k_next = p.mu_k[nbh];
       }
       const int nl = n0 + T - 1;  // the item's last block
+      // Tile ping-pong: the last block is not folded into F'; the epilogue forms
+      // O = (F' ratio + acc e) v_scale / (255 L') from both, with the fold's arithmetic.
+      float e_last = 1.0f, r_last = 1.0f, L_fin;
+      bool last_only = false;  // the item's only block: O = acc v_scale / (255 l)
       if constexpr (C::kTilePP) {
-        // The item's last block: its P.V, then its fold.
         if (!wait_warp(&bars[Bar::pvdone(qt)], nl & 1, abort_flag)) {
           alive = false;
           break;
         }
-        tc_fence_after();
-        fold_block(T - 1, m_run, lt_prev);
-        tmem_st_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars[Bar::folddone(qt)]);
-      } else if (!wait_warp(&bars[Bar::folddone(nl & 1)], (nl >> 1) & 1, abort_flag)) {
-        alive = false;
-        break;
+        last_only = (T == 1);
+        float Lp = 0.0f;
+        if (!last_only) {
+          const float2 lm = s_Lm[r];
+          Lp = lm.x;
+          e_last = ex2_approx((m_run - lm.y) * kLog2e);
+          if (e_last > 1.8446744e19f) {
+            r_last = 1.0f / e_last;
+            e_last = 1.0f;
+          }
+        }
+        L_fin = last_only ? lt_prev : __fmaf_rn(lt_prev, e_last, Lp * r_last);
+      } else {
+        if (!wait_warp(&bars[Bar::folddone(nl & 1)], (nl >> 1) & 1, abort_flag)) {
+          alive = false;
+          break;
+        }
+        L_fin = 0.0f;
       }
       tc_fence_after();
-      const float inv_l = 1.0f / (255.0f * s_Lm[r].x);
+      if constexpr (!C::kTilePP) L_fin = s_Lm[r].x;
+      const float inv_l = 1.0f / (255.0f * L_fin);
       const int esz = (p.o_dt == BA_F32) ? 4 : 2;
       const bool vec = ((d * esz) & 15) == 0;
       // Block ping-pong: each group writes half of the row's channels; tile ping-pong: all.
@@ -1133,9 +1146,25 @@ __global__ void __launch_bounds__(Cfg<DP, BK>::kThreads, 1)
       for (int g0 = 0; g0 < kChan; g0 += 8) {
         const int c0 = (C::kTilePP ? 0 : grp * DH) + g0;  // eight channels at a time
         uint32_t f[8];
-        tmem_ld_cols<8>(aF + c0, f);
-        tmem_ld_wait();
-        reg_fence8(f);
+        if constexpr (C::kTilePP) {
+          uint32_t a[8];
+          tmem_ld_cols<8>(aAcc + c0, a);
+          if (!last_only) tmem_ld_cols<8>(aF + c0, f);
+          tmem_ld_wait();
+          reg_fence8(a);
+          if (!last_only) reg_fence8(f);
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const float av = __fadd_rn(__uint_as_float(a[k] + kMagicBits), -kMagic);
+            const float fo = last_only ? 0.0f : (r_last != 1.0f ? __fmul_rn(__uint_as_float(f[k]), r_last)
+                                                                : __uint_as_float(f[k]));
+            f[k] = __float_as_uint(last_only ? av : __fmaf_rn(av, e_last, fo));
+          }
+        } else {
+          tmem_ld_cols<8>(aF + c0, f);
+          tmem_ld_wait();
+          reg_fence8(f);
+        }
         float val[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
