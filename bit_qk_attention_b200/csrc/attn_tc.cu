@@ -30,8 +30,8 @@
 //   * Each block's product is weighted by e_j = exp(m_j - m_ref) against a per-row reference
 //     maximum: the output sum F' = sum_j acc_j e_j (tensor memory, fp32) and the softmax sum
 //     L' = sum_j l_j e_j give O = F' v_scale / (255 L'), the blockwise online softmax's result.
-//     A block's |acc| <= 255 * 127 * 128 < 2^22 converts exactly through the bit pattern of
-//     1.5 * 2^23.
+//     Each P.V accumulates onto the bit pattern of 1.5 * 2^23, so a block's product
+//     (|acc| <= 255 * 127 * 128 < 2^22) reads directly as the float 1.5 * 2^23 + acc.
 //   * Near-tie codes are made exact: where a code of the fast exponential could differ from the
 //     definition's (two roundings of 255 P~, scaled by 1 -+ eps, disagree), the key's
 //     double-precision d = s - m is compared with a host-computed threshold table. This check
@@ -639,7 +639,7 @@ __global__ void __launch_bounds__(Cfg<DP, BK>::kThreads, 1)
 #pragma unroll
           for (int kk = 0; kk < BN / 32; ++kk)
             mma_i8_ts(tmem + C::tAcc(q), tmem + C::tS(q, 0) + 8 * kk, smem_desc(vbase + 512 * kk, 128, 2048),
-                      idesc_pv, kk > 0 ? 1u : 0u);
+                      idesc_pv, 1u);
           tc_commit(&bars[Bar::pvdone(q)]);
           if (q == 1) tc_commit(&bars[Bar::kvempty(n % S)]);  // the last reader of stage n
           return true;
@@ -660,7 +660,7 @@ __global__ void __launch_bounds__(Cfg<DP, BK>::kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < BN / 32; ++kk)
           mma_i8_ts(tmem + C::tAcc(0), tmem + C::tS(0, j & 1) + 8 * kk, smem_desc(vbase + 512 * kk, 128, 2048),
-                    idesc_pv, kk > 0 ? 1u : 0u);
+                    idesc_pv, 1u);
         tc_commit(&bars[Bar::pvdone(j & 1)]);
         tc_commit(&bars[Bar::kvempty(j % S)]);
         if (j + 2 < nblocks && !qk(j + 2)) break;
@@ -703,6 +703,18 @@ __global__ void __launch_bounds__(Cfg<DP, BK>::kThreads, 1)
     bool alive = true;
     float mu_q_next = 0.0f, mu_k_next = 0.0f;  // mu of the item about to start (loaded one item ahead)
     int n0 = 0;  // index, counted across items, of the item's first key block
+    // The P.V accumulator holds the bit pattern of 1.5 * 2^23 whenever no product is in it: every
+    // P.V accumulates onto it, so a block's s32 result reads directly as the float
+    // 1.5 * 2^23 + acc (|acc| < 2^22), and whoever reads a product restores the pattern. Each
+    // group sets its rows once here (tile ping-pong: its own tile; block ping-pong: group 0 for
+    // the shared accumulator), before its first P arrival.
+    uint32_t kmag[32];
+#pragma unroll
+    for (int k = 0; k < 32; ++k) kmag[k] = kMagicBits;
+    if (C::kTilePP || grp == 0) {
+#pragma unroll
+      for (int c = 0; c < DP; c += 16) tmem_st_cols<16>(aAcc + c, kmag);
+    }
     for (int it = 0; it < n_items && alive; ++it, n0 += T) {
       int64_t bh;
       int q0;
@@ -797,9 +809,8 @@ __global__ void __launch_bounds__(Cfg<DP, BK>::kThreads, 1)
             const float2 e2 = make_float2(e, e), rt2 = make_float2(ratio, ratio);
 #pragma unroll
             for (int k = 0; k < G; k += 2) {
-              const float2 a2 = __fadd2_rn(
-                  make_float2(__uint_as_float(a[k] + kMagicBits), __uint_as_float(a[k + 1] + kMagicBits)),
-                  make_float2(-kMagic, -kMagic));
+              const float2 a2 = __fadd2_rn(make_float2(__uint_as_float(a[k]), __uint_as_float(a[k + 1])),
+                                           make_float2(-kMagic, -kMagic));
               float2 f2;
               if (FIRST) {
                 f2 = a2;
@@ -811,10 +822,13 @@ __global__ void __launch_bounds__(Cfg<DP, BK>::kThreads, 1)
               f[k] = __float_as_uint(f2.x);
               f[k + 1] = __float_as_uint(f2.y);
             }
-            if (c0 + G <= DP)
+            if (c0 + G <= DP) {
               tmem_st_cols<G>(aF + c0, f);
-            else
+              tmem_st_cols<G>(aAcc + c0, kmag);
+            } else {
               tmem_st_cols<16>(aF + c0, f);
+              tmem_st_cols<16>(aAcc + c0, kmag);
+            }
           }
         };
         if (tb == 0)
@@ -1155,11 +1169,12 @@ __global__ void __launch_bounds__(Cfg<DP, BK>::kThreads, 1)
           if (!last_only) reg_fence8(f);
 #pragma unroll
           for (int k = 0; k < 8; ++k) {
-            const float av = __fadd_rn(__uint_as_float(a[k] + kMagicBits), -kMagic);
+            const float av = __fadd_rn(__uint_as_float(a[k]), -kMagic);
             const float fo = last_only ? 0.0f : (r_last != 1.0f ? __fmul_rn(__uint_as_float(f[k]), r_last)
                                                                 : __uint_as_float(f[k]));
             f[k] = __float_as_uint(last_only ? av : __fmaf_rn(av, e_last, fo));
           }
+          tmem_st_cols<8>(aAcc + c0, kmag);
         } else {
           tmem_ld_cols<8>(aF + c0, f);
           tmem_ld_wait();
